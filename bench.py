@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of the frame-wise GDN scan (libgdn) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload rollout] [--impl libgdn|reference]
+
+One step is one gdn_frame_scan over the whole workload (every head, every
+frame) with the inputs already resident in HBM. The inputs (10.4 GB for the
+961-frame rollout) are far larger than L2, so no L2 flush is needed between
+steps. With N > 1 (torchrun) every rank scans its own copy of the workload on
+its own GPU: the heads are independent, there is no collective on the data
+path, and the scaling is weak. Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle (the only reference this
+method has) on a bounded sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from frame_wise_gated_scan_b200 import inputs  # noqa: E402
+
+METRIC = "GDN frames·heads/s on the 961×880-token rollout (B=1, H=32, D=64, T=961, S=880, bf16)"
+UNIT = "frames·heads/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="rollout", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="libgdn", choices=["libgdn", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "frame_wise_gated_scan_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"scan_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        loaded = [float(r[1]) for r in rows if float(r[3]) > 200.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+def device_inputs(wl, device):
+    import torch
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    shape = (wl.B, wl.H, wl.T, wl.S, wl.D)
+    q = torch.empty(shape, dtype=dt, device=device)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    g = torch.empty((wl.B, wl.H, wl.T), dtype=torch.float32, device=device)
+    be = torch.empty_like(g)
+    for b, h, qq, kk, vv, gg, bb in inputs.iter_heads_packed(wl):
+        for dst, src in ((q, qq), (k, kk), (v, vv)):
+            t = torch.from_numpy(src.view(np.int16)).view(torch.bfloat16) if wl.dtype == "bf16" \
+                else torch.from_numpy(src)
+            dst[b, h].copy_(t)
+        g[b, h].copy_(torch.from_numpy(gg))
+        be[b, h].copy_(torch.from_numpy(bb))
+    return q, k, v, g, be
+
+
+def cpu_baseline(wl, seconds: float):
+    """The float64 oracle, as it stands, on whole heads of the workload until
+    the time budget is spent (at least one head's first frames)."""
+    from oracle import gdn_scan_ref
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    done_frames = 0
+    heads = 0
+    t_total = 0.0
+    chunk = min(wl.T, 64)
+    b = h = 0
+    while t_total < seconds:
+        T = min(chunk, wl.T)
+        q, k, v, g, be = inputs.head(wl, b, h, T)
+        t0 = time.perf_counter()
+        gdn_scan_ref(q, k, v, g, be)
+        t_total += time.perf_counter() - t0
+        done_frames += T
+        heads += 1
+        h = (h + 1) % wl.H
+        if h == 0:
+            b = (b + 1) % wl.B
+    return {"value": done_frames / t_total, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} runs of the float64 oracle over the first {chunk} frames of one "
+                      f"head each (S={wl.S}, D={wl.D}), {t_total:.1f} s of CPU time; "
+                      f"numpy BLAS threads={cores}"}
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    cb_seconds = max(1.0, min(args.cpu_seconds, 60.0))
+    # each step: the oracle over one head for a bounded number of frames
+    T = min(wl.T, 24)
+    from oracle import gdn_scan_ref
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        h = i % wl.H
+        q, k, v, g, be = inputs.head(wl, 0, h, T)
+        t0 = time.perf_counter()
+        gdn_scan_ref(q, k, v, g, be)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            per_step.append(dt)
+    total = sum(per_step)
+    value = args.steps * T / total
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, workload shapes)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T, "S": wl.S,
+                   "step": f"float64 oracle over {T} frames of one head"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {T} frames of one head (S={wl.S}, D={wl.D})"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del cb_seconds
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    wl = inputs.WORKLOADS[args.workload]
+    if wl.name == "step":
+        wl = inputs.WORKLOADS["rollout"]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+    import torch
+    import torch.distributed as dist
+    from frame_wise_gated_scan_b200 import gdn
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+
+    kern, ctas = gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D)
+    q, k, v, g, be = device_inputs(wl, device)
+    out = torch.empty_like(q)
+    st = torch.empty((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        gdn.frame_scan(q, k, v, g, be, None, out=out, state_out=st)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if gdn.device_status() != 0:
+        raise RuntimeError("a device-side wait ran out during warm-up")
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launch_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            launch_ev[i][0].record(stream)
+            step()
+            launch_ev[i][1].record(stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    launch_ms = [a.elapsed_time(b) for a, b in launch_ev]
+    if gdn.device_status() != 0:
+        raise RuntimeError("a device-side wait ran out during the timed steps")
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    units = wl.heads * wl.T
+    value = units * args.steps * world / (max_ms / 1e3)
+    mean_launch_s = statistics.mean(launch_ms) / 1e3
+    alg_bytes = inputs.algorithmic_bytes(wl)
+    achieved = alg_bytes / mean_launch_s / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # End to end through the public API on pinned host buffers.
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hg, hb = (x.cpu().pin_memory() for x in (q, k, v, g, be))
+        del q, k, v
+        torch.cuda.empty_cache()
+        staging = {}
+        out_h = torch.empty(hq.shape, dtype=hq.dtype, pin_memory=True)
+        st_h = torch.empty(st.shape, dtype=torch.float32, pin_memory=True)
+        gdn.frame_scan_host(hq, hk, hv, hg, hb, staging=staging, out_host=out_h, state_host=st_h)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            gdn.frame_scan_host(hq, hk, hv, hg, hb, staging=staging, out_host=out_h,
+                                state_host=st_h)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb))
+        d2h = out_h.numel() * out_h.element_size() + st_h.numel() * 4
+        e2e = {"value": units * args.e2e_steps * world / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": args.e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; rollout recipe: Q,V ~ N(0,1), K rows L2-normalised, "
+                "gamma ~ U(.95,1), beta ~ U(.2,1))",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T, "S": wl.S,
+                   "global_batch": wl.B * world, "seq_len": wl.T * wl.S,
+                   "parallelism": f"replicas x{world} (heads independent, no collective)",
+                   "kernel": {1: "simt", 2: "tcgen05"}[kern], "ctas_per_head": ctas,
+                   "l2": "inputs larger than L2 (10.4 GB read per step), no flush"},
+        "gpu_launches": args.steps,
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": recorded_traffic(wl.name),
+                     "algorithmic_bytes_per_launch": alg_bytes},
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+// C-ABI entry points of libgdn (declared in include/gdn.h): argument checks,
+// the key scale, kernel choice, launch.
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "gdn.h"
+#include "gdn_internal.h"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// [lo, hi) byte ranges overlap?
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Kernel override for debugging: GDN_IMPL=simt forces the CUDA-core kernel.
+int forced_kernel() {
+  static int cached = -1;
+  if (cached < 0) {
+    const char* e = getenv("GDN_IMPL");
+    cached = (e && strcmp(e, "simt") == 0) ? GDN_KERNEL_SIMT : 0;
+  }
+  return cached;
+}
+
+int check_sizes(int B, int H, int T, int S, int D) {
+  if (B < 1 || H < 1 || T < 1 || S < 1) return GDN_ERR_SHAPE;
+  if (D != 32 && D != 64 && D != 128) return GDN_ERR_UNSUPPORTED_D;
+  const double elems = (double)B * H * T * S * D;
+  if (elems > 9.0e18 / 4.0) return GDN_ERR_SHAPE;
+  if ((long long)B * H > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  return GDN_OK;
+}
+
+int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
+  const int f = forced_kernel();
+  const int tc = (f == GDN_KERNEL_SIMT) ? 0 : gdn::tc_ctas_per_head(B, H, T, S, D);
+  if (tc > 0) {
+    *ctas = tc;
+    return GDN_KERNEL_TC;
+  }
+  *ctas = 1;
+  return GDN_KERNEL_SIMT;
+}
+
+int run(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
+        const float* state_in, float* state_out, void* out, int B, int H, int T, int S, int D,
+        void* stream, int elt_bytes) {
+  const int sz = check_sizes(B, H, T, S, D);
+  if (sz != GDN_OK) return sz;
+  if (!q || !k || !v || !gamma || !beta || !out) return GDN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(gamma, 4) ||
+      !aligned(beta, 4))
+    return GDN_ERR_ALIGN;
+  const size_t n = (size_t)B * H * T * S * D * elt_bytes;
+  const size_t ns = (size_t)B * H * D * D * sizeof(float);
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) ||
+      overlap(out, n, state_in, ns) || overlap(out, n, state_out, ns))
+    return GDN_ERR_ALIAS;
+  if (state_in && state_out && state_in != state_out && overlap(state_in, ns, state_out, ns))
+    return GDN_ERR_ALIAS;
+
+  gdn::Problem p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gamma = gamma;
+  p.beta = beta;
+  p.state_in = state_in;
+  p.state_out = state_out;
+  p.out = out;
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.S = S;
+  p.D = D;
+  p.key_scale = (float)(1.0 / sqrt((double)D * (double)S));
+  p.stream = static_cast<cudaStream_t>(stream);
+
+  cudaError_t err;
+  if (elt_bytes == 4) {
+    err = gdn::launch_simt_f32(p);
+  } else {
+    int ctas = 1;
+    const int kern = choose_kernel(B, H, T, S, D, &ctas);
+    err = (kern == GDN_KERNEL_TC) ? gdn::launch_tc_bf16(p, ctas) : gdn::launch_simt_bf16(p);
+  }
+  return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_frame_scan(const void* q, const void* k, const void* v, const float* gamma,
+                   const float* beta, const float* state_in, float* state_out, void* out, int B,
+                   int H, int T, int S, int D, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 2);
+}
+
+int gdn_frame_step(const void* q, const void* k, const void* v, const float* gamma,
+                   const float* beta, const float* state_in, float* state_out, void* out, int B,
+                   int H, int S, int D, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 2);
+}
+
+int gdn_frame_scan_f32(const float* q, const float* k, const float* v, const float* gamma,
+                       const float* beta, const float* state_in, float* state_out, float* out,
+                       int B, int H, int T, int S, int D, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 4);
+}
+
+int gdn_frame_step_f32(const float* q, const float* k, const float* v, const float* gamma,
+                       const float* beta, const float* state_in, float* state_out, float* out,
+                       int B, int H, int S, int D, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 4);
+}
+
+int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head) {
+  const int sz = check_sizes(B, H, T, S, D);
+  if (sz != GDN_OK) return sz;
+  if (!kernel || !ctas_per_head) return GDN_ERR_NULL;
+  *kernel = choose_kernel(B, H, T, S, D, ctas_per_head);
+  return GDN_OK;
+}
+
+int gdn_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+  unsigned int st = 0;
+  if (gdn::tc_read_status(&st) != cudaSuccess) return GDN_ERR_CUDA;
+  return st ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_NULL: return "a required pointer is NULL";
+    case GDN_ERR_SHAPE: return "B, H, T and S must be >= 1 and the sizes must fit in 64 bits";
+    case GDN_ERR_UNSUPPORTED_D: return "D must be 32, 64 or 128";
+    case GDN_ERR_ALIGN: return "q, k, v, out and the states must be 16-byte aligned; gamma and beta 4-byte aligned";
+    case GDN_ERR_CUDA: return "a CUDA call failed";
+    case GDN_ERR_TIMEOUT: return "a device-side wait ran out; outputs of that call are incomplete";
+    case GDN_ERR_ALIAS: return "out overlaps an input or a state buffer";
+    default: return "unknown gdn_status";
+  }
+}
+
+int gdn_version(void) {
+  return GDN_VERSION_MAJOR * 10000 + GDN_VERSION_MINOR * 100 + GDN_VERSION_PATCH;
+}
+
+}  // extern "C"

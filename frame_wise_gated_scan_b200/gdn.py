@@ -1,0 +1,209 @@
+"""Python binding of libgdn (include/gdn.h): argument marshalling only.
+
+Every step of the recurrence runs in the library's CUDA kernels. This module
+checks tensors, allocates outputs with torch (device memory is the caller's
+side of the ABI), passes raw pointers and the current CUDA stream, and turns
+a negative status into GdnError. There is no fallback: without the built
+library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
+
+KERNEL_SIMT = 1
+KERNEL_TC = 2
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions include/gdn.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)
+
+
+def lib() -> ctypes.CDLL:
+    """The in-tree libgdn.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdn.so not built at {LIB_PATH}; run "
+                               "python -m frame_wise_gated_scan_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+        scan_args = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
+        step_args = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, vp]
+        for name, args in (("gdn_frame_scan", scan_args), ("gdn_frame_scan_f32", scan_args),
+                           ("gdn_frame_step", step_args), ("gdn_frame_step_f32", step_args)):
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = i
+        L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
+        L.gdn_plan.restype = i
+        L.gdn_device_status.argtypes = []
+        L.gdn_device_status.restype = i
+        L.gdn_status_string.argtypes = [i]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return lib().gdn_version()
+
+
+def plan(B: int, H: int, T: int, S: int, D: int) -> tuple[int, int]:
+    """(kernel id, CTAs per head) a bf16 call with these sizes would use."""
+    k, c = ctypes.c_int(), ctypes.c_int()
+    st = lib().gdn_plan(B, H, T, S, D, ctypes.byref(k), ctypes.byref(c))
+    if st != 0:
+        raise GdnError(st, "gdn_plan")
+    return k.value, c.value
+
+
+def device_status() -> int:
+    """Synchronizes and returns the library's device status (0 = no wait ran out)."""
+    return lib().gdn_device_status()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(t, name, dtype, shape, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state):
+    if q.dim() != (4 if step else 5):
+        raise ValueError("q must be [B,H,S,D] for a step, [B,H,T,S,D] for a scan")
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("tensors must be CUDA tensors (use frame_scan_host for host buffers)")
+    dt = q.dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bfloat16 or float32")
+    if step:
+        B, H, S, D = q.shape
+        T = 1
+        gshape = (B, H)
+    else:
+        B, H, T, S, D = q.shape
+        gshape = (B, H, T)
+    for name, t in (("k", k), ("v", v)):
+        _check(t, name, dt, q.shape, device)
+    _check(gamma, "gamma", torch.float32, gshape, device)
+    _check(beta, "beta", torch.float32, gshape, device)
+    if state_in is not None:
+        _check(state_in, "state_in", torch.float32, (B, H, D, D), device)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", dt, q.shape, device)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+    elif state_out is not None:
+        _check(state_out, "state_out", torch.float32, (B, H, D, D), device)
+    L = lib()
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in),
+            _ptr(state_out), _ptr(out), B, H]
+    if not step:
+        args.append(T)
+    args += [S, D, _stream_handle(device)]
+    if step:
+        fn = L.gdn_frame_step if dt == torch.bfloat16 else L.gdn_frame_step_f32
+    else:
+        fn = L.gdn_frame_scan if dt == torch.bfloat16 else L.gdn_frame_scan_f32
+    with torch.cuda.device(device):
+        st = fn(*args)
+    if st != 0:
+        raise GdnError(st, fn.__name__)
+    return out, state_out
+
+
+def frame_scan(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
+               want_state=True):
+    """T frames per head. q, k, v: [B,H,T,S,D] bf16 or fp32 CUDA tensors;
+    gamma, beta: [B,H,T] fp32; state_in: [B,H,D,D] fp32 or None (zero).
+    Returns (out, state_out); state_out is None if want_state is False and
+    none was given."""
+    return _call(False, q, k, v, gamma, beta, state_in, out, state_out, want_state)
+
+
+def frame_step(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
+               want_state=True):
+    """One frame per head (chunk-causal rollout). q, k, v: [B,H,S,D];
+    gamma, beta: [B,H]. state_out may be state_in (in-place carry)."""
+    return _call(True, q, k, v, gamma, beta, state_in, out, state_out, want_state)
+
+
+def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,
+                    staging=None, out_host=None, state_host=None):
+    """End-to-end call on HOST tensors: copies the inputs to the GPU, runs the
+    scan there, copies out and the final state back, and waits for them.
+
+    Pass pinned tensors for asynchronous copies. `staging` may hold reusable
+    device buffers (a dict filled on the first call) and out_host/state_host
+    reusable pinned outputs."""
+    device = torch.device(device or "cuda")
+    stream = stream or torch.cuda.current_stream(device)
+    staging = {} if staging is None else staging
+    with torch.cuda.device(device), torch.cuda.stream(stream):
+        def dev(name, t):
+            if t is None:
+                return None
+            buf = staging.get(name)
+            if buf is None or buf.shape != t.shape or buf.dtype != t.dtype:
+                buf = torch.empty(t.shape, dtype=t.dtype, device=device)
+                staging[name] = buf
+            buf.copy_(t, non_blocking=True)
+            return buf
+        dq, dk, dv = dev("q", q), dev("k", k), dev("v", v)
+        dg, db, ds = dev("gamma", gamma), dev("beta", beta), dev("state_in", state_in)
+        if "out" not in staging or staging["out"].shape != q.shape or staging["out"].dtype != q.dtype:
+            staging["out"] = torch.empty(q.shape, dtype=q.dtype, device=device)
+        D = q.shape[-1]
+        sshape = (q.shape[0], q.shape[1], D, D)
+        if "state_out" not in staging or tuple(staging["state_out"].shape) != sshape:
+            staging["state_out"] = torch.empty(sshape, dtype=torch.float32, device=device)
+        frame_scan(dq, dk, dv, dg, db, ds, out=staging["out"], state_out=staging["state_out"])
+        if out_host is None:
+            out_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        if state_host is None:
+            state_host = torch.empty(sshape, dtype=torch.float32, pin_memory=True)
+        out_host.copy_(staging["out"], non_blocking=True)
+        state_host.copy_(staging["state_out"], non_blocking=True)
+        stream.synchronize()
+    return out_host, state_host

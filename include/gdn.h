@@ -1,0 +1,121 @@
+/*
+ * libgdn: the frame-wise Gated DeltaNet (GDN) scan on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("NVIDIA Apresenta SANA-WM: Um Modelo de Mundo de Larga
+ * Escala ...", acheiumaia.com.br, section "A Arquitetura: Quatro Decisoes de
+ * Design Centrais", item "1. Atencao Linear Hibrida com Gated DeltaNet"):
+ * every latent frame of S spatial tokens is one recurrent step on a constant
+ * D x D state per head, with a decay gate gamma, a delta-rule correction and
+ * keys scaled by 1/sqrt(D*S). Per head and frame t, with K_t, Q_t, V_t of
+ * shape S x D, s = 1/sqrt(D*S) and M of shape D x D:
+ *
+ *     W   = (s K_t) M_{t-1}
+ *     R   = V_t - gamma_t W
+ *     M_t = gamma_t M_{t-1} + beta_t (s K_t)^T R
+ *     O_t = Q_t M_t
+ *
+ * Layouts (all row-major, contiguous, element strides implied by the sizes):
+ *   q, k, v, out   [B][H][T][S][D]   scan;  [B][H][S][D] step (T = 1)
+ *   gamma, beta    [B][H][T] float   scan;  [B][H] float      step
+ *   state_in/out   [B][H][D][D] float; element [i][j]: i = key dim, j = value dim
+ * Keys are passed unscaled: the library applies s = 1/sqrt(D*S) itself.
+ * Gates are used as given (not clamped or validated; NaN propagates).
+ *
+ * Pointers: every array pointer is a DEVICE pointer of the current CUDA
+ * device. The caller owns every buffer; the library keeps no pointer after a
+ * call returns and allocates no device memory. q, k, v, out, state_in and
+ * state_out must be 16-byte aligned; gamma and beta 4-byte aligned.
+ * state_in == NULL means M_0 = 0. state_out == NULL means the final state is
+ * not written. state_in may equal state_out (the update is then in place);
+ * out must not overlap q, k, v or the states.
+ *
+ * Ordering: work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ * default stream) and the call returns without waiting for it. Arguments
+ * are checked first, on the host; on any error nothing is enqueued and a
+ * negative gdn_status is returned.
+ *
+ * Device-side waits inside the kernels are bounded. A kernel whose wait runs
+ * out stops early, leaves its outputs incomplete and records
+ * GDN_ERR_TIMEOUT in a device status word; read it with gdn_device_status().
+ */
+#ifndef LIBGDN_GDN_H_
+#define LIBGDN_GDN_H_
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_VERSION_MAJOR 1
+#define GDN_VERSION_MINOR 0
+#define GDN_VERSION_PATCH 0
+
+typedef enum gdn_status {
+  GDN_OK = 0,
+  GDN_ERR_NULL = -1,            /* q, k, v, gamma, beta or out is NULL */
+  GDN_ERR_SHAPE = -2,           /* B, H, T or S < 1, or a size overflows 64 bits */
+  GDN_ERR_UNSUPPORTED_D = -3,   /* D not in {32, 64, 128} */
+  GDN_ERR_ALIGN = -4,           /* a pointer breaks the alignment rules above */
+  GDN_ERR_CUDA = -5,            /* a CUDA runtime or driver call failed */
+  GDN_ERR_TIMEOUT = -6,         /* a device-side wait ran out (from gdn_device_status) */
+  GDN_ERR_ALIAS = -7            /* out overlaps an input or a state buffer */
+} gdn_status;
+
+/* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
+ * Arithmetic: fp32 accumulation on tcgen05 tensor cores, fp32 state kept on
+ * chip across all T frames, out rounded to bf16 (round to nearest even). */
+GDN_API int gdn_frame_scan(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int T, int S, int D, void* stream);
+
+/* One bf16 frame (T = 1) for chunk-causal rollout: the state is read from
+ * state_in and written to state_out, which may be the same buffer, so a
+ * caller can carry it across calls. Same arithmetic as gdn_frame_scan; a chain
+ * of steps gives the same result as one scan over the same frames. */
+GDN_API int gdn_frame_step(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int S, int D, void* stream);
+
+/* float32 variants: q, k, v, out are float; every operation runs in fp32 on
+ * CUDA cores (FFMA), in the definition's order (W, then R, then K^T R). */
+GDN_API int gdn_frame_scan_f32(const float* q, const float* k, const float* v,
+                       const float* gamma, const float* beta,
+                       const float* state_in, float* state_out, float* out,
+                       int B, int H, int T, int S, int D, void* stream);
+
+GDN_API int gdn_frame_step_f32(const float* q, const float* k, const float* v,
+                       const float* gamma, const float* beta,
+                       const float* state_in, float* state_out, float* out,
+                       int B, int H, int S, int D, void* stream);
+
+/* Which kernel a bf16 call with these sizes runs, without running it.
+ * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head
+ * (the thread-block cluster size, 1 for the CUDA-core kernel).
+ * Returns GDN_OK or the error the call itself would return for the sizes. */
+#define GDN_KERNEL_SIMT 1   /* CUDA-core kernel, one CTA per 16 state columns */
+#define GDN_KERNEL_TC 2     /* tcgen05 kernel, a cluster of CTAs per head */
+GDN_API int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head);
+
+/* Synchronizes the current device, then returns GDN_ERR_TIMEOUT if any kernel
+ * since the last call recorded a wait that ran out (and clears the record),
+ * GDN_ERR_CUDA if the synchronize failed, else GDN_OK. */
+GDN_API int gdn_device_status(void);
+
+/* Static text for a gdn_status value. Never NULL. */
+GDN_API const char* gdn_status_string(int status);
+
+/* GDN_VERSION_MAJOR * 10000 + GDN_VERSION_MINOR * 100 + GDN_VERSION_PATCH */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBGDN_GDN_H_ */

@@ -1,0 +1,177 @@
+"""CUDA path against the float64 oracle, element by element, through the C ABI.
+
+Tolerances (relative Frobenius error per frame and head, and per head for the
+final state): 1e-5 for fp32 inputs, 2e-2 for bf16 inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from frame_wise_gated_scan_b200 import gdn, inputs
+from gpu_util import (TOL_BF16, TOL_F32, assert_close, device_workload, oracle_head, to_np64)
+
+pytestmark = pytest.mark.gpu
+
+_cache = {}
+
+
+def workload_on_device(name, T=None):
+    key = (name, T)
+    if key not in _cache:
+        _cache.clear()           # keep one large workload resident at a time
+        _cache[key] = device_workload(inputs.WORKLOADS[name], T)
+    return _cache[key]
+
+
+def _scan_and_compare(wl, heads=None, T=None, tol=None, state_in=None):
+    q, k, v, g, be = device_workload(wl, T)
+    st_dev = None if state_in is None else torch.from_numpy(state_in).cuda()
+    out, st = gdn.frame_scan(q, k, v, g, be, st_dev)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    tol = tol or (TOL_F32 if wl.dtype == "f32" else TOL_BF16)
+    heads = heads or [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    worst = 0.0
+    for b, h in heads:
+        ro, rs = oracle_head(wl, b, h, T, None if state_in is None else state_in[b, h])
+        e, _ = assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, tol, f"{wl.name} b{b} h{h}")
+        worst = max(worst, e)
+    return worst
+
+
+def test_tiny_fp32():
+    _scan_and_compare(inputs.WORKLOADS["tiny"])
+
+
+def test_tiny_fp32_with_state():
+    wl = inputs.WORKLOADS["tiny"]
+    _scan_and_compare(wl, state_in=inputs.state(wl))
+
+
+def test_tiny_fp32_step_chain_equals_scan():
+    wl = inputs.WORKLOADS["tiny"]
+    q, k, v, g, be = device_workload(wl)
+    out, st = gdn.frame_scan(q, k, v, g, be)
+    state = torch.zeros((wl.B, wl.H, wl.D, wl.D), device="cuda")
+    for t in range(wl.T):
+        o_t, _ = gdn.frame_step(q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                v[:, :, t].contiguous(), g[:, :, t].contiguous(),
+                                be[:, :, t].contiguous(), state, state_out=state)
+        assert torch.equal(o_t, out[:, :, t])
+    assert torch.equal(state, st)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("S", [1, 63, 64, 65, 127, 128, 129, 200])
+def test_bf16_shapes(S, D):
+    wl = inputs.Workload(f"shape_s{S}_d{D}", 1, 3, D, 3, S, "bf16", 100 + S + D, "gauss", "tiny")
+    _scan_and_compare(wl)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("S", [1, 65, 200])
+def test_fp32_shapes(S, D):
+    wl = inputs.Workload(f"f32_s{S}_d{D}", 1, 2, D, 2, S, "f32", 300 + S + D, "gauss", "tiny")
+    _scan_and_compare(wl)
+
+
+@pytest.mark.parametrize("T", [1, 2, 8])
+def test_bf16_frames_and_state(T):
+    wl = inputs.Workload(f"t{T}", 2, 3, 64, T, 880, "bf16", 400 + T, "l2", "rollout")
+    _scan_and_compare(wl, state_in=inputs.state(wl, scale=0.5))
+
+
+def test_short_config_all_heads():
+    _scan_and_compare(inputs.WORKLOADS["short"])
+
+
+@pytest.mark.slow
+def test_rollout_full_size_sampled_heads():
+    wl = inputs.WORKLOADS["rollout"]
+    q, k, v, g, be = workload_on_device("rollout")
+    out, st = gdn.frame_scan(q, k, v, g, be)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert torch.isfinite(out).all() and torch.isfinite(st).all()
+    for b, h in [(0, 0), (0, 17), (0, 31)]:
+        ro, rs = oracle_head(wl, b, h)
+        assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16, f"rollout h{h}")
+
+
+@pytest.mark.slow
+def test_step_chain_rollout_matches_scan():
+    """961 gdn_frame_step calls with the state carried in place equal one scan."""
+    wl = inputs.WORKLOADS["step"]
+    q, k, v, g, be = workload_on_device("rollout")
+    out, st = gdn.frame_scan(q, k, v, g, be)
+    state = torch.zeros((wl.B, wl.H, wl.D, wl.D), device="cuda")
+    o_step = torch.empty((wl.B, wl.H, wl.S, wl.D), dtype=torch.bfloat16, device="cuda")
+    mismatched = 0
+    for t in range(wl.T):
+        gdn.frame_step(q[:, :, t].contiguous(), k[:, :, t].contiguous(), v[:, :, t].contiguous(),
+                       g[:, :, t].contiguous(), be[:, :, t].contiguous(), state, out=o_step,
+                       state_out=state)
+        mismatched += int(not torch.equal(o_step, out[:, :, t]))
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    e = float((state - st).norm() / st.norm())
+    assert e <= 1e-6, f"step-chain final state vs scan: {e:.3e}"
+    ro, rs = oracle_head(wl, 0, 5)
+    assert_close(to_np64(out[0, 5]), ro, to_np64(state[0, 5]), rs, TOL_BF16, "step chain h5")
+    print(f"step chain: state rel diff {e:.3e}, frames with differing out: {mismatched}")
+
+
+@pytest.mark.slow
+def test_stress_full_size_sampled_heads():
+    wl = inputs.WORKLOADS["stress"]
+    q, k, v, g, be = workload_on_device("stress")
+    out, st = gdn.frame_scan(q, k, v, g, be)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert torch.isfinite(out).all() and torch.isfinite(st).all(), "stress: NaN/Inf"
+    for b, h in [(0, 0), (3, 15)]:
+        ro, rs = oracle_head(wl, b, h)
+        assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16, f"stress b{b} h{h}")
+
+
+def test_null_state_means_zero_and_state_out_optional():
+    wl = inputs.Workload("nulls", 1, 2, 64, 2, 130, "bf16", 7, "gauss", "tiny")
+    q, k, v, g, be = device_workload(wl)
+    z = torch.zeros((1, 2, 64, 64), device="cuda")
+    o1, s1 = gdn.frame_scan(q, k, v, g, be, None)
+    o2, s2 = gdn.frame_scan(q, k, v, g, be, z)
+    o3, s3 = gdn.frame_scan(q, k, v, g, be, None, want_state=False)
+    torch.cuda.synchronize()
+    assert s3 is None
+    assert torch.equal(o1, o2) and torch.equal(s1, s2) and torch.equal(o1, o3)
+
+
+def test_in_place_step_state():
+    wl = inputs.Workload("inplace", 1, 4, 64, 1, 300, "bf16", 8, "gauss", "tiny")
+    q, k, v, g, be = device_workload(wl)
+    m0 = torch.from_numpy(inputs.state(wl)).cuda()
+    ref_o, ref_s = gdn.frame_step(q[:, :, 0].contiguous(), k[:, :, 0].contiguous(),
+                                  v[:, :, 0].contiguous(), g[:, :, 0].contiguous(),
+                                  be[:, :, 0].contiguous(), m0.clone())
+    st = m0.clone()
+    o, _ = gdn.frame_step(q[:, :, 0].contiguous(), k[:, :, 0].contiguous(), v[:, :, 0].contiguous(),
+                          g[:, :, 0].contiguous(), be[:, :, 0].contiguous(), st, state_out=st)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(st, ref_s)
+
+
+def test_bad_arguments_launch_nothing():
+    q = torch.zeros((1, 1, 1, 8, 48), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones((1, 1, 1), device="cuda")
+    with pytest.raises(gdn.GdnError) as ei:
+        gdn.frame_scan(q, q.clone(), q.clone(), g, g.clone())
+    assert ei.value.status == -3
+
+
+def test_host_buffers_end_to_end():
+    wl = inputs.Workload("host", 1, 2, 64, 3, 200, "bf16", 9, "gauss", "tiny")
+    q, k, v, g, be = device_workload(wl)
+    ref_o, ref_s = gdn.frame_scan(q, k, v, g, be)
+    hq, hk, hv, hg, hb = (x.cpu().pin_memory() for x in (q, k, v, g, be))
+    o, s = gdn.frame_scan_host(hq, hk, hv, hg, hb)
+    assert torch.equal(o, ref_o.cpu()) and torch.equal(s, ref_s.cpu())
