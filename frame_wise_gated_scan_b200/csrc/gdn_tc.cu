@@ -1,13 +1,847 @@
-// tcgen05 kernel of the frame-wise GDN scan (placeholder: takes no sizes yet).
+// tcgen05 kernel of the frame-wise Gated DeltaNet scan, bf16 inputs, D = 64.
+//
+// The update ("NVIDIA Apresenta SANA-WM ...", acheiumaia.com.br, section
+// "A Arquitetura", item "1. Atencao Linear Hibrida com Gated DeltaNet"), per
+// head and frame t with s = 1/sqrt(D*S):
+//     W = (sK) M,  R = V - gamma W,  M' = gamma M + beta (sK)^T R,  O = Q M'.
+// Since (sK)^T R = s K^T V - gamma s^2 (K^T K) M, the same update reads
+//     M' = gamma M + A' M + c,   A' = -gamma beta s^2 G,  G = K^T K,  c = beta s K^T V.
+// G and K^T V depend on the frame's keys and values only, not on the state,
+// so the two S-long contractions that build them run ahead of the
+// recurrence; the only work on the frame-to-frame critical path is the
+// D x D x D product A' M. The read-out O = Q M' follows behind it.
+//
+// Work split. One thread-block cluster of P CTAs per head (P = 1, 2 or 4):
+//  * frames are dealt round-robin: CTA r owns frames r, r+P, ...; for its
+//    frames it streams K, V, Q (TMA, 128-row tiles, 128-byte swizzle), forms
+//    [G; (K^T V)^T] = [K V]^T K on the tensor cores, turns it into A' (bf16
+//    hi + lo) and c, and writes them into every CTA's shared memory;
+//  * the value columns of the state never mix, so CTA r runs the recurrence
+//    for its NC = 64/P state columns on every frame: its fp32 slice of M
+//    stays in registers across all T frames, and its bf16 hi/lo copy is the
+//    MMA operand of the next frame;
+//  * each CTA sends its slice of M_t to the owner of frame t, which computes
+//    O_t = Q_t M_t (M in bf16 hi + lo, two MMAs) and stores it with TMA.
+// Warp roles (512 threads): 0 K/V loader, 1 Q loader, 2 MMA issuer (and TMEM
+// allocation), 3 idle, 4-7 recurrence epilogue, 8-11 A'/c epilogue,
+// 12-15 output epilogue.
+//
+// Every wait is bounded (kTimeoutNs). A wait that runs out sets the device
+// status word and an abort flag in every CTA of the cluster; the other roles
+// then stop, in-flight copies and MMAs are drained, and the kernel returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdlib.h>
+
 #include "gdn_internal.h"
+#include "sm100_ptx.h"
 
 namespace gdn {
 
 __device__ unsigned int g_tc_status = 0;
 
-int tc_ctas_per_head(int, int, int, int, int) { return 0; }
+namespace {
 
-cudaError_t launch_tc_bf16(const Problem&, int) { return cudaErrorNotSupported; }
+using namespace ptx;
+
+constexpr uint64_t kTimeoutNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
+constexpr int kThreads = 512;
+constexpr int kD = 64;
+constexpr int kTile = 128;                                      // rows per tile
+constexpr uint32_t kTileBytes = kTile * kD * 2;                 // 16 KB
+constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+
+// Status codes recorded in g_tc_status (bit per waiting role).
+enum : uint32_t {
+  kStKvLoad = 1u << 0, kStQLoad = 1u << 1, kStMma = 1u << 2, kStChain = 1u << 3,
+  kStProd = 1u << 4, kStOut = 1u << 5, kStDrain = 1u << 6, kStMoEmpty = 1u << 7,
+  kStAcEmpty = 1u << 8
+};
+
+template <int P>
+struct Layout {
+  static constexpr int NC = kD / P;                  // state columns per CTA
+  static constexpr int NAC = P < 2 ? 2 : P;          // transition-operand slots
+  static constexpr int NKV = 2;
+  static constexpr int NQ = 2;
+  static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
+  static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
+  static constexpr uint32_t C_BYTES = kD * NC * 4;                  // c slice, fp32 [64][NC]
+  static constexpr uint32_t AC_SLOT = align1k(2 * AP_BYTES + C_BYTES);
+  static constexpr uint32_t RW = NC * 2;                            // bytes per slice row
+  static constexpr uint32_t SBO = 8 * RW;                           // 8-row group stride
+  static constexpr uint32_t MS_PART = kD * RW;                      // slice, hi or lo
+  static constexpr uint32_t MS_BUF = align1k(2 * MS_PART);
+  static constexpr uint32_t MO_PART = kD * kD * 2;                  // full M, hi or lo
+  static constexpr uint32_t MO_BUF = 2 * MO_PART;
+  static constexpr uint32_t SWZ_CODE = NC == 64 ? 2u : (NC == 32 ? 4u : 6u);
+  static constexpr int SWZ_BITS = NC == 64 ? 3 : (NC == 32 ? 2 : 1);
+
+  static constexpr uint32_t OFF_KV = 0;
+  static constexpr uint32_t OFF_Q = OFF_KV + NKV * KV_SLOT;
+  static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
+  static constexpr uint32_t OFF_MS = OFF_AC + NAC * AC_SLOT;
+  static constexpr uint32_t OFF_MO = OFF_MS + 2 * MS_BUF;
+  static constexpr uint32_t OFF_BAR = OFF_MO + 2 * MO_BUF;
+  // barrier indices (8 bytes each)
+  static constexpr int B_KV_FULL = 0;
+  static constexpr int B_KV_EMPTY = B_KV_FULL + NKV;
+  static constexpr int B_Q_FULL = B_KV_EMPTY + NKV;
+  static constexpr int B_Q_EMPTY = B_Q_FULL + NQ;
+  static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;
+  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;
+  static constexpr int B_GB_FULL = B_AC_EMPTY + NAC;
+  static constexpr int B_GB_FREE = B_GB_FULL + 2;
+  static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
+  static constexpr int B_M_READY = B_CHAIN_DONE + 1;
+  static constexpr int B_MO_FULL = B_M_READY + 1;
+  static constexpr int B_MO_EMPTY = B_MO_FULL + 2;                  // [P][2]
+  static constexpr int B_O_FULL = B_MO_EMPTY + 2 * P;
+  static constexpr int B_O_FREE = B_O_FULL + 2;
+  static constexpr int B_DRAIN = B_O_FREE + 2;
+  static constexpr int B_STAGE = B_DRAIN + 1;   // [2] output tile staged by the 4 warps
+  static constexpr int NBAR = B_STAGE + 2;
+  static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
+  static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
+  static constexpr uint32_t BYTES = OFF_ABORT + 16;
+  static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;              // base alignment slack
+
+  // TMEM columns (each region 128 lanes)
+  static constexpr uint32_t T_GB = 0;        // 2 x 64: [G; (K^T V)^T] accumulators
+  static constexpr uint32_t T_O = 128;       // 2 x 64: output tile accumulators
+  static constexpr uint32_t T_CHAIN = 256;   // NC columns, M = 64 layout
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+static_assert(Layout<4>::SMEM_ALLOC <= 232448, "shared memory budget (P=4)");
+static_assert(Layout<2>::SMEM_ALLOC <= 232448, "shared memory budget (P=2)");
+static_assert(Layout<1>::SMEM_ALLOC <= 232448, "shared memory budget (P=1)");
+
+struct TcParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_o;
+  const float* gamma;
+  const float* beta;
+  const float* state_in;
+  float* state_out;
+  unsigned int* status;
+  int T;
+  int S;
+  int ntile;
+  float s;     // key scale 1/sqrt(D*S)
+  float s2;    // its square
+};
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
+// `row_bytes` long and grouped by 8 rows, with the matching swizzle (the
+// layout TMA writes with CU_TENSOR_MAP_SWIZZLE_{32,64,128}B and the tcgen05
+// descriptors read): bits [4, 4+b) of the offset are XORed with bits [7, 7+b).
+__device__ __forceinline__ uint32_t swz_off(uint32_t row, uint32_t chunk, uint32_t row_bytes,
+                                            int bits) {
+  const uint32_t off = (row >> 3) * (8 * row_bytes) + (row & 7) * row_bytes + chunk * 16;
+  return off ^ (((off >> 7) & ((1u << bits) - 1)) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): 8 values -> two 16-byte chunks.
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(x[e]);
+    h[e] = __bfloat162float(b);
+    l[e] = x[e] - h[e];
+  }
+  hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
+                  pack_bf16x2(h[6], h[7]));
+  lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]),
+                  pack_bf16x2(l[6], l[7]));
+}
+
+struct Ctl {
+  uint32_t abort_addr;    // local shared address of the abort flag
+  unsigned int* status;
+  int P;
+};
+
+__device__ __forceinline__ bool aborted(const Ctl& c) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(c.abort_addr) : "memory");
+  return v != 0;
+}
+
+__device__ __noinline__ void raise_abort(const Ctl& c, uint32_t code) {
+  atomicOr(c.status, code);
+  for (int q = 0; q < c.P; ++q) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa(c.abort_addr, q)), "r"(1u)
+                 : "memory");
+  }
+  fence_acq_rel_cluster();
+}
+
+// Bounded wait on a local mbarrier phase. False if the kernel is aborting or
+// the wait ran out (then the abort is raised with `code`).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c,
+                                         uint32_t code) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (aborted(c)) return false;
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      raise_abort(c, code);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, and on
+// success every lane observes the completed phase itself (acquire).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl& c,
+                                          uint32_t code) {
+  uint32_t ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, c, code) ? 1u : 0u;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) {
+    for (int i = 0; i < 1024 && !mbar_try(bar, parity); ++i) {
+    }
+  }
+  return ok != 0;
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight copies).
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      atomicOr(c.status, kStDrain);
+      return;
+    }
+  }
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ TcParams p) {
+  using L = Layout<P>;
+  constexpr int NC = L::NC;
+  constexpr int NAC = L::NAC;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;         // 1 KB aligned base, same in every CTA
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int bh = blockIdx.x / P;
+  const int T = p.T;
+  const int ntile = p.ntile;
+  const int nown = (T > (int)rank) ? (T - (int)rank + P - 1) / P : 0;   // frames this CTA owns
+
+  auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * i; };
+  auto kv_slot = [&](int i) -> uint32_t { return sb + L::OFF_KV + i * L::KV_SLOT; };
+  auto q_slot = [&](int i) -> uint32_t { return sb + L::OFF_Q + i * kTileBytes; };
+  auto ac_slot = [&](int i) -> uint32_t { return sb + L::OFF_AC + i * L::AC_SLOT; };
+  auto ms_buf = [&](int i) -> uint32_t { return sb + L::OFF_MS + i * L::MS_BUF; };
+  auto mo_buf = [&](int i) -> uint32_t { return sb + L::OFF_MO + i * L::MO_BUF; };
+  const uint32_t tmem_ptr = sb + L::OFF_TMEM_PTR;
+  Ctl ctl{sb + L::OFF_ABORT, p.status, P};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NKV; ++i) {
+      mbar_init(bar(L::B_KV_FULL + i), 1);
+      mbar_init(bar(L::B_KV_EMPTY + i), 1);
+    }
+    for (int i = 0; i < L::NQ; ++i) {
+      mbar_init(bar(L::B_Q_FULL + i), 1);
+      mbar_init(bar(L::B_Q_EMPTY + i), 1);
+    }
+    for (int i = 0; i < NAC; ++i) {
+      mbar_init(bar(L::B_AC_FULL + i), 4);          // the producer's 4 epilogue warps
+      mbar_init(bar(L::B_AC_EMPTY + i), 4 * P);     // 4 recurrence warps of every CTA
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_GB_FULL + i), 1);
+      mbar_init(bar(L::B_GB_FREE + i), 4);
+      mbar_init(bar(L::B_MO_FULL + i), 4 * P);
+      mbar_init(bar(L::B_O_FULL + i), 1);
+      mbar_init(bar(L::B_O_FREE + i), 4);
+    }
+    for (int i = 0; i < 2 * P; ++i) mbar_init(bar(L::B_MO_EMPTY + i), 1);
+    mbar_init(bar(L::B_CHAIN_DONE), 1);
+    mbar_init(bar(L::B_M_READY), 4);
+    mbar_init(bar(L::B_DRAIN), 1);
+    mbar_init(bar(L::B_STAGE + 0), 4);
+    mbar_init(bar(L::B_STAGE + 1), 4);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+    prefetch_tmap(&p.tm_o);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_ptr, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();   // every CTA's barriers exist before any remote arrive
+  uint32_t tmem;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_ptr) : "memory");
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ K/V loader (own frames)
+    int it = 0;
+    for (int j = 0; j < nown; ++j) {
+      const int f = (int)rank + j * P;
+      bool ok = true;
+      for (int i = 0; i < ntile; ++i, ++it) {
+        const int slot = it % L::NKV;
+        if (!wait_bar(bar(L::B_KV_EMPTY + slot), ((it / L::NKV) & 1) ^ 1, ctl, kStKvLoad)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::B_KV_FULL + slot), 2 * kTileBytes);
+        tma_load_3d(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kTile, bh * T + f);
+        tma_load_3d(kv_slot(slot) + kTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0, i * kTile,
+                    bh * T + f);
+      }
+      if (!ok) break;
+    }
+    for (int k = it - 1; k >= 0 && k >= it - L::NKV; --k)
+      drain_bar(bar(L::B_KV_FULL + k % L::NKV), (k / L::NKV) & 1, ctl);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ Q loader (own frames)
+    int it = 0;
+    for (int j = 0; j < nown; ++j) {
+      const int f = (int)rank + j * P;
+      bool ok = true;
+      for (int i = 0; i < ntile; ++i, ++it) {
+        const int slot = it % L::NQ;
+        if (!wait_bar(bar(L::B_Q_EMPTY + slot), ((it / L::NQ) & 1) ^ 1, ctl, kStQLoad)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::B_Q_FULL + slot), kTileBytes);
+        tma_load_3d(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, i * kTile, bh * T + f);
+      }
+      if (!ok) break;
+    }
+    for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
+      drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t id_chain = idesc_bf16(64, NC, 0, 1);    // A' K-major, M slice MN-major
+    constexpr uint32_t id_gb = idesc_bf16(128, 64, 1, 1);      // [K V]^T and K, both MN-major
+    constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);       // Q K-major, M MN-major
+    int t = 0;                         // next frame of the recurrence
+    int gj = 0, gi = 0, kvit = 0;      // [G; b^T] stream: own frame, tile, ring counter
+    int oj = 0, oi = 0, qit = 0, on = 0;
+    uint64_t t0 = globaltimer_ns();
+    while (t < T || gj < nown || oj < nown) {
+      bool progressed = false;
+      if (t < T && mbar_test(bar(L::B_M_READY), t & 1) &&
+          mbar_test(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1)) {
+        tc_fence_after();
+        const uint32_t ac = ac_slot(t % NAC);
+        const uint32_t mb = ms_buf((t + 1) & 1);                 // slice of M_{t-1}
+        const uint32_t dt = tmem + L::T_CHAIN;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
+          const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
+          const uint64_t bH = smem_desc(mb + kk * 2 * L::SBO, L::MS_PART, L::SBO, L::SWZ_CODE);
+          const uint64_t bL = smem_desc(mb + L::MS_PART + kk * 2 * L::SBO, L::MS_PART, L::SBO,
+                                        L::SWZ_CODE);
+          mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
+          mma_bf16(dt, aH, bL, id_chain, 1u);
+          mma_bf16(dt, aL, bH, id_chain, 1u);
+        }
+        mma_commit(bar(L::B_CHAIN_DONE));
+        ++t;
+        progressed = true;
+      }
+      if (gj < nown) {
+        const int slot = kvit % L::NKV;
+        const int b = gj & 1;
+        if (mbar_test(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1) &&
+            (gi > 0 || mbar_test(bar(L::B_GB_FREE + b), ((gj >> 1) & 1) ^ 1))) {
+          tc_fence_after();
+          const uint32_t kv = kv_slot(slot);
+          const uint32_t dg = tmem + L::T_GB + 64 * b;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
+            const uint64_t bd = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
+            mma_bf16(dg, a, bd, id_gb, (gi > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_KV_EMPTY + slot));
+          if (gi == ntile - 1) {
+            mma_commit(bar(L::B_GB_FULL + b));
+            gi = 0;
+            ++gj;
+          } else {
+            ++gi;
+          }
+          ++kvit;
+          progressed = true;
+        }
+      }
+      if (oj < nown) {
+        const int slot = qit % L::NQ;
+        const int ob = on & 1;
+        const int u = oj & 1;
+        if (mbar_test(bar(L::B_Q_FULL + slot), (qit / L::NQ) & 1) &&
+            mbar_test(bar(L::B_O_FREE + ob), ((on >> 1) & 1) ^ 1) &&
+            (oi > 0 || mbar_test(bar(L::B_MO_FULL + u), (oj >> 1) & 1))) {
+          tc_fence_after();
+          const uint32_t qt = q_slot(slot);
+          const uint32_t mo = mo_buf(u);
+          const uint32_t dO = tmem + L::T_O + 64 * ob;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = smem_desc(qt + kk * 32, 16, 1024, 2);
+            const uint64_t bH = smem_desc(mo + kk * 2 * L::SBO, kD * L::RW, L::SBO, L::SWZ_CODE);
+            const uint64_t bL = smem_desc(mo + L::MO_PART + kk * 2 * L::SBO, kD * L::RW, L::SBO,
+                                          L::SWZ_CODE);
+            mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
+            mma_bf16(dO, a, bL, id_o, 1u);
+          }
+          mma_commit(bar(L::B_O_FULL + ob));
+          ++qit;
+          ++on;
+          if (++oi == ntile) {
+            oi = 0;
+            ++oj;
+          }
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        t0 = globaltimer_ns();
+      } else {
+        if (aborted(ctl)) break;
+        if (globaltimer_ns() - t0 > kTimeoutNs) {
+          raise_abort(ctl, kStMma);
+          break;
+        }
+      }
+    }
+    mma_commit(bar(L::B_DRAIN));
+    drain_bar(bar(L::B_DRAIN), 0, ctl);
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------ recurrence epilogue
+    const int qd = warp & 3;
+    const int row = qd * 16 + lane;            // M = 64 accumulator: rows 16qd.. in lanes 32qd..
+    const bool act = lane < 16;
+    const int j0 = (int)rank * NC;
+    float m[NC];                               // fp32 state, row `row`, columns j0..j0+NC
+#pragma unroll
+    for (int jj = 0; jj < NC; ++jj)
+      m[jj] = (act && p.state_in) ? p.state_in[((size_t)bh * kD + row) * kD + j0 + jj] : 0.f;
+    if (act) {
+#pragma unroll
+      for (int c = 0; c < NC / 8; ++c) {       // M_{-1} = M_0 into operand buffer 1
+        uint4 h, l;
+        split8(&m[8 * c], h, l);
+        const uint32_t off = swz_off(row, c, L::RW, L::SWZ_BITS);
+        st_shared_v4(ms_buf(1) + off, h);
+        st_shared_v4(ms_buf(1) + L::MS_PART + off, l);
+      }
+    }
+    fence_proxy_async_cta();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::B_M_READY));
+    const float* gam = p.gamma + (size_t)bh * T;
+    float g_next = __ldg(gam);
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const float g = g_next;
+      if (t + 1 < T) g_next = __ldg(gam + t + 1);
+      const int s = t % NAC;
+      if (!warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain) ||
+          !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + (act ? row : 0) * NC * 4;
+      const uint32_t mbuf = ms_buf(t & 1);
+#pragma unroll
+      for (int c16 = 0; c16 < NC / 16; ++c16) {
+        uint32_t d[16];
+        tmem_ld16(tmem + L::T_CHAIN + 16 * c16 + ((uint32_t)(qd * 32) << 16), d);
+        tmem_wait_ld();
+        if (act) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 cv = ld_shared_f4(crow + 64 * c16 + 16 * c4);
+            float* mm = &m[16 * c16 + 4 * c4];
+            mm[0] = fmaf(g, mm[0], __uint_as_float(d[4 * c4 + 0])) + cv.x;
+            mm[1] = fmaf(g, mm[1], __uint_as_float(d[4 * c4 + 1])) + cv.y;
+            mm[2] = fmaf(g, mm[2], __uint_as_float(d[4 * c4 + 2])) + cv.z;
+            mm[3] = fmaf(g, mm[3], __uint_as_float(d[4 * c4 + 3])) + cv.w;
+          }
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            uint4 h, l;
+            split8(&m[16 * c16 + 8 * h8], h, l);
+            const uint32_t off = swz_off(row, 2 * c16 + h8, L::RW, L::SWZ_BITS);
+            st_shared_v4(mbuf + off, h);
+            st_shared_v4(mbuf + L::MS_PART + off, l);
+          }
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_cta();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(L::B_M_READY));                       // M_t slice ready, TMEM free
+        if (t + NAC < T) mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + s), (t + NAC) % P));
+      }
+      // Slice of M_t to the CTA that owns frame t, for its read-out.
+      const int dst = t % P;
+      const int jo = t / P;
+      const int u = jo & 1;
+      if (!warp_wait(bar(L::B_MO_EMPTY + 2 * dst + u), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty)) {
+        ok = false;
+        break;
+      }
+      if (act) {
+        const uint32_t base = mapa(mo_buf(u) + rank * (kD * L::RW), dst);
+#pragma unroll
+        for (int c = 0; c < NC / 8; ++c) {
+          uint4 h, l;
+          split8(&m[8 * c], h, l);
+          const uint32_t off = swz_off(row, c, L::RW, L::SWZ_BITS);
+          st_cluster_v4(base + off, h);
+          st_cluster_v4(base + L::MO_PART + off, l);
+        }
+      }
+      fence_proxy_async_cluster();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
+    }
+    if (ok && act && p.state_out) {
+#pragma unroll
+      for (int jj = 0; jj < NC; ++jj) p.state_out[((size_t)bh * kD + row) * kD + j0 + jj] = m[jj];
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------ A' and c from [G; (K^T V)^T]
+    const int qd = warp & 3;
+    const int lrow = qd * 32 + lane;           // accumulator row = TMEM lane
+    int waits[NAC];
+#pragma unroll
+    for (int i = 0; i < NAC; ++i) waits[i] = 0;
+    const float* gam = p.gamma + (size_t)bh * T;
+    const float* bet = p.beta + (size_t)bh * T;
+    for (int j = 0; j < nown; ++j) {
+      const int f = (int)rank + j * P;
+      const int b = j & 1;
+      const float g = __ldg(gam + f);
+      const float be = __ldg(bet + f);
+      if (!warp_wait(bar(L::B_GB_FULL + b), (j >> 1) & 1, ctl, kStProd)) break;
+      tc_fence_after();
+      uint32_t v[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r16[16];
+        tmem_ld16(tmem + L::T_GB + 64 * b + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_GB_FREE + b));
+      const int s = f % NAC;
+      if (f >= NAC) {
+        int w = 0;
+#pragma unroll
+        for (int i = 0; i < NAC; ++i)
+          if (i == s) w = waits[i];
+        if (!warp_wait(bar(L::B_AC_EMPTY + s), w & 1, ctl, kStAcEmpty)) break;
+#pragma unroll
+        for (int i = 0; i < NAC; ++i)
+          if (i == s) waits[i] += 1;
+      }
+      const uint32_t slot = ac_slot(s);
+      if (lrow < kD) {
+        // row lrow of A' = -gamma beta s^2 G, as bf16 hi + lo, K-major, 128-byte swizzle
+        const float coef = -g * be * p.s2;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = coef * __uint_as_float(v[8 * c + e]);
+          uint4 h, l;
+          split8(x, h, l);
+          const uint32_t off = swz_off(lrow, c, 128, 3);
+          for (int q = 0; q < P; ++q) {
+            st_cluster_v4(mapa(slot + off, q), h);
+            st_cluster_v4(mapa(slot + L::AP_BYTES + off, q), l);
+          }
+        }
+      } else {
+        // column (lrow - 64) of c = beta s K^T V, to the CTA that owns that state column
+        const int jc = lrow - kD;
+        const uint32_t dst = mapa(slot + 2 * L::AP_BYTES + (jc % NC) * 4, jc / NC);
+        const float coef = be * p.s;
+#pragma unroll
+        for (int i = 0; i < kD; ++i) st_cluster_f32(dst + i * NC * 4, coef * __uint_as_float(v[i]));
+      }
+      fence_proxy_async_cluster();
+      __syncwarp();
+      if (lane == 0) {
+        for (int q = 0; q < P; ++q) mbar_arrive_cluster(mapa(bar(L::B_AC_FULL + s), q));
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------ output tiles: TMEM -> bf16 -> TMA store
+    const int qd = warp & 3;
+    const int lrow = qd * 32 + lane;
+    const bool leader = (warp == 12 && lane == 0);
+    int n = 0;
+    bool ok = true;
+    for (int j = 0; j < nown && ok; ++j) {
+      const int f = (int)rank + j * P;
+      for (int i = 0; i < ntile; ++i, ++n) {
+        const int ob = n & 1;
+        if (!warp_wait(bar(L::B_O_FULL + ob), (n >> 1) & 1, ctl, kStOut)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r16[16];
+          tmem_ld16(tmem + L::T_O + 64 * ob + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_O_FREE + ob));
+        const int slot = n % L::NQ;                  // the Q tile this output came from
+        const uint32_t tile = q_slot(slot);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+          w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+          w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+          w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+          st_shared_v4(tile + swz_off(lrow, c, 128, 3), w);
+        }
+        fence_proxy_async_cta();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_STAGE + (n & 1)));
+        if (leader) {
+          if (!wait_bar(bar(L::B_STAGE + (n & 1)), (n >> 1) & 1, ctl, kStOut)) {
+            ok = false;
+            break;
+          }
+          tma_store_3d(&p.tm_o, tile, 0, i * kTile, bh * T + f);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar(L::B_Q_EMPTY + slot));
+          if (i == ntile - 1)
+            for (int q = 0; q < P; ++q)
+              mbar_arrive_cluster(mapa(bar(L::B_MO_EMPTY + 2 * rank + (j & 1)), q));
+        }
+      }
+    }
+    if (leader) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // no CTA leaves while a peer may still write into its shared memory
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [B*H*T][S][64] bf16 viewed as a 3-D tensor (64, S, B*H*T); 64 x 128 x 1 boxes with
+// the 128-byte swizzle. Rows past S inside a frame read as zero and are not stored.
+bool make_map(CUtensorMap* m, const void* base, int S, long long frames) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S, (cuuint64_t)frames};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S * kD * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int P>
+const void* kernel_ptr() {
+  return reinterpret_cast<const void*>(&gdn_tc_kernel<P>);
+}
+
+template <int P>
+cudaError_t prepare() {
+  static bool done = false;
+  static cudaError_t err = cudaSuccess;
+  if (!done) {
+    err = cudaFuncSetAttribute(kernel_ptr<P>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)Layout<P>::SMEM_ALLOC);
+    done = true;
+  }
+  return err;
+}
+
+// Clusters of P CTAs that can be resident at once on the current device, or
+// -1 if there is no usable device (host-only planning). Cached per device.
+template <int P>
+int resident_clusters() {
+  static int cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (have[dev]) return cache[dev];
+  int n = -1;
+  if (prepare<P>() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(P * 64, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Layout<P>::SMEM_ALLOC;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, gdn_tc_kernel<P>, &cfg) != cudaSuccess) n = -1;
+  }
+  cudaGetLastError();
+  cache[dev] = n;
+  have[dev] = true;
+  return n;
+}
+
+unsigned int* status_word() {
+  static unsigned int* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_tc_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<unsigned int*>(ptr);
+  }
+  return cache[dev];
+}
+
+template <int P>
+cudaError_t launch_p(const Problem& pr) {
+  cudaError_t e = prepare<P>();
+  if (e != cudaSuccess) return e;
+  TcParams p;
+  const long long frames = (long long)pr.B * pr.H * pr.T;
+  if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames) ||
+      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames))
+    return cudaErrorInvalidValue;
+  unsigned int* status = status_word();
+  if (!status) return cudaErrorInvalidDevice;
+  p.gamma = pr.gamma;
+  p.beta = pr.beta;
+  p.state_in = pr.state_in;
+  p.state_out = pr.state_out;
+  p.status = status;
+  p.T = pr.T;
+  p.S = pr.S;
+  p.ntile = (pr.S + kTile - 1) / kTile;
+  p.s = pr.key_scale;
+  const double sd = 1.0 / ((double)kD * (double)pr.S);
+  p.s2 = (float)sd;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(pr.B * pr.H * P), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<P>::SMEM_ALLOC;
+  cfg.stream = pr.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<P>, p);
+}
+
+}  // namespace
+
+int tc_ctas_per_head(int B, int H, int T, int S, int D) {
+  if (D != kD) return 0;
+  const long long heads = (long long)B * H;
+  if (heads * (long long)T >= (1ll << 31) || (long long)S * kD * 2 >= (1ll << 40)) return 0;
+  if (heads * 4 > (1ll << 31) - 1) return 0;
+  // Tuning override: GDN_TC_CTAS=1|2|4 forces the cluster size.
+  if (const char* e = getenv("GDN_TC_CTAS")) {
+    const int v = atoi(e);
+    if (v == 1 || v == 2 || v == 4) return v;
+  }
+  if (T == 1) return 1;
+  // Largest cluster size whose clusters all fit on the device at once.
+  const int c4 = resident_clusters<4>();
+  const int c2 = resident_clusters<2>();
+  const int sms = 148;
+  const long long fit4 = c4 >= 0 ? c4 : sms / 4;
+  const long long fit2 = c2 >= 0 ? c2 : sms / 2;
+  if (heads <= fit4) return 4;
+  if (heads <= fit2) return 2;
+  return 1;
+}
+
+cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head) {
+  switch (ctas_per_head) {
+    case 1: return launch_p<1>(p);
+    case 2: return launch_p<2>(p);
+    case 4: return launch_p<4>(p);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t tc_read_status(unsigned int* status) {
   unsigned int zero = 0;
