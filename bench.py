@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="run only the first N frames of the workload (profiling captures)")
     return ap.parse_args()
 
 
@@ -236,6 +238,8 @@ def main():
     wl = inputs.WORKLOADS[args.workload]
     if wl.name == "step":
         wl = inputs.WORKLOADS["rollout"]
+    if args.frames:
+        wl = wl.with_(T=min(args.frames, wl.T))
     if args.impl == "reference":
         run_reference(args, wl)
         return

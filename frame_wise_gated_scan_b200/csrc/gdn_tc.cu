@@ -21,10 +21,10 @@
 //    stays in registers across all T frames, and its bf16 hi/lo copy is the
 //    MMA operand of the next frame;
 //  * each CTA sends its slice of M_t to the owner of frame t, which computes
-//    O_t = Q_t M_t (M in bf16 hi + lo, two MMAs) and stores it with TMA.
+//    O_t = Q_t M_t (M in bf16 hi + lo, two MMAs) and stores it.
 // Warp roles (512 threads): 0 K/V loader, 1 Q loader, 2 MMA issuer (and TMEM
-// allocation), 3 idle, 4-7 recurrence epilogue, 8-11 A'/c epilogue,
-// 12-15 output epilogue.
+// allocation), 3 forwarder (state slices to frame owners), 4-7 recurrence
+// epilogue, 8-11 A'/c epilogue, 12-15 output epilogue.
 //
 // Every wait is bounded (kTimeoutNs). A wait that runs out sets the device
 // status word and an abort flag in every CTA of the cluster; the other roles
@@ -62,9 +62,10 @@ enum : uint32_t {
 template <int P>
 struct Layout {
   static constexpr int NC = kD / P;                  // state columns per CTA
-  static constexpr int NAC = P < 2 ? 2 : P;          // transition-operand slots
-  static constexpr int NKV = 2;
-  static constexpr int NQ = 2;
+  static constexpr int NAC = P == 4 ? 3 : 2;         // transition-operand slots
+  static constexpr int NKV = 2;                      // K/V tile pairs in flight
+  static constexpr int NQ = P == 1 ? 2 : 3;          // Q tiles in flight
+  static constexpr int NMS = P == 1 ? 2 : 4;         // state-slice ring (MMA operand + outbox)
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
   static constexpr uint32_t C_BYTES = kD * NC * 4;                  // c slice, fp32 [64][NC]
@@ -82,7 +83,7 @@ struct Layout {
   static constexpr uint32_t OFF_Q = OFF_KV + NKV * KV_SLOT;
   static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
   static constexpr uint32_t OFF_MS = OFF_AC + NAC * AC_SLOT;
-  static constexpr uint32_t OFF_MO = OFF_MS + 2 * MS_BUF;
+  static constexpr uint32_t OFF_MO = OFF_MS + NMS * MS_BUF;
   static constexpr uint32_t OFF_BAR = OFF_MO + 2 * MO_BUF;
   // barrier indices (8 bytes each)
   static constexpr int B_KV_FULL = 0;
@@ -100,8 +101,9 @@ struct Layout {
   static constexpr int B_O_FULL = B_MO_EMPTY + 2 * P;
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;
-  static constexpr int B_STAGE = B_DRAIN + 1;   // [2] output tile staged by the 4 warps
-  static constexpr int NBAR = B_STAGE + 2;
+  static constexpr int B_MS_FULL = B_DRAIN + 1;                     // [NMS] slice written
+  static constexpr int B_MS_FREE = B_MS_FULL + NMS;                 // [NMS] slice forwarded
+  static constexpr int NBAR = B_MS_FREE + NMS;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -127,6 +129,7 @@ struct TcParams {
   const float* beta;
   const float* state_in;
   float* state_out;
+  uint16_t* out;           // bf16 bit patterns
   unsigned int* status;
   int T;
   int S;
@@ -263,21 +266,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     for (int i = 0; i < NAC; ++i) {
       mbar_init(bar(L::B_AC_FULL + i), 4);          // the producer's 4 epilogue warps
-      mbar_init(bar(L::B_AC_EMPTY + i), 4 * P);     // 4 recurrence warps of every CTA
+      mbar_init(bar(L::B_AC_EMPTY + i), P);         // the forwarder of every CTA
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
       mbar_init(bar(L::B_GB_FREE + i), 4);
-      mbar_init(bar(L::B_MO_FULL + i), 4 * P);
+      mbar_init(bar(L::B_MO_FULL + i), P);          // the forwarder of every CTA
       mbar_init(bar(L::B_O_FULL + i), 1);
       mbar_init(bar(L::B_O_FREE + i), 4);
     }
     for (int i = 0; i < 2 * P; ++i) mbar_init(bar(L::B_MO_EMPTY + i), 1);
+    for (int i = 0; i < L::NMS; ++i) {
+      mbar_init(bar(L::B_MS_FULL + i), 4);
+      mbar_init(bar(L::B_MS_FREE + i), 1);
+    }
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
     mbar_init(bar(L::B_DRAIN), 1);
-    mbar_init(bar(L::B_STAGE + 0), 4);
-    mbar_init(bar(L::B_STAGE + 1), 4);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
   }
@@ -353,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           mbar_test(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1)) {
         tc_fence_after();
         const uint32_t ac = ac_slot(t % NAC);
-        const uint32_t mb = ms_buf((t + 1) & 1);                 // slice of M_{t-1}
+        const uint32_t mb = ms_buf((t + L::NMS - 1) % L::NMS);   // slice of M_{t-1}
         const uint32_t dt = tmem + L::T_CHAIN;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -416,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
             mma_bf16(dO, a, bL, id_o, 1u);
           }
+          mma_commit(bar(L::B_Q_EMPTY + slot));
           mma_commit(bar(L::B_O_FULL + ob));
           ++qit;
           ++on;
@@ -438,6 +444,32 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     mma_commit(bar(L::B_DRAIN));
     drain_bar(bar(L::B_DRAIN), 0, ctl);
+  } else if (warp == 3) {
+    // ------------------------------------------------ forwarder: state slices to frame owners
+    for (int t = 0; t < T; ++t) {
+      const int slot = t % L::NMS;
+      if (!warp_wait(bar(L::B_MS_FULL + slot), (t / L::NMS) & 1, ctl, kStChain)) break;
+      // The recurrence has read c_t and its MMA has read A'_t: release the slot.
+      if (lane == 0 && t + NAC < T)
+        mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + t % NAC), (t + NAC) % P));
+      const int dst = t % P;
+      const int jo = t / P;
+      const int u = jo & 1;
+      if (!warp_wait(bar(L::B_MO_EMPTY + 2 * dst + u), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty))
+        break;
+      const uint32_t src = ms_buf(slot);
+      const uint32_t dhi = mapa(mo_buf(u) + rank * L::MS_PART, dst);
+      for (uint32_t off = lane * 16; off < L::MS_PART; off += 512) {
+        st_cluster_v4(dhi + off, ld_shared_u4(src + off));
+        st_cluster_v4(dhi + L::MO_PART + off, ld_shared_u4(src + L::MS_PART + off));
+      }
+      fence_proxy_async_cluster();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
+        mbar_arrive(bar(L::B_MS_FREE + slot));
+      }
+    }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------ recurrence epilogue
     const int qd = warp & 3;
@@ -449,13 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int jj = 0; jj < NC; ++jj)
       m[jj] = (act && p.state_in) ? p.state_in[((size_t)bh * kD + row) * kD + j0 + jj] : 0.f;
     if (act) {
+      const uint32_t b0 = ms_buf(L::NMS - 1);  // M_{-1} = M_0, read by the first MMA
 #pragma unroll
-      for (int c = 0; c < NC / 8; ++c) {       // M_{-1} = M_0 into operand buffer 1
+      for (int c = 0; c < NC / 8; ++c) {
         uint4 h, l;
         split8(&m[8 * c], h, l);
         const uint32_t off = swz_off(row, c, L::RW, L::SWZ_BITS);
-        st_shared_v4(ms_buf(1) + off, h);
-        st_shared_v4(ms_buf(1) + L::MS_PART + off, l);
+        st_shared_v4(b0 + off, h);
+        st_shared_v4(b0 + L::MS_PART + off, l);
       }
     }
     fence_proxy_async_cta();
@@ -468,14 +501,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
+      const int slot = t % L::NMS;
       if (!warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain) ||
-          !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain)) {
+          !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
+          (t >= L::NMS &&
+           !warp_wait(bar(L::B_MS_FREE + slot), ((t / L::NMS) & 1) ^ 1, ctl, kStChain))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + (act ? row : 0) * NC * 4;
-      const uint32_t mbuf = ms_buf(t & 1);
+      const uint32_t mbuf = ms_buf(slot);
 #pragma unroll
       for (int c16 = 0; c16 < NC / 16; ++c16) {
         uint32_t d[16];
@@ -505,31 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(L::B_M_READY));                       // M_t slice ready, TMEM free
-        if (t + NAC < T) mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + s), (t + NAC) % P));
+        mbar_arrive(bar(L::B_M_READY));        // M_t slice is the next MMA operand; TMEM free
+        mbar_arrive(bar(L::B_MS_FULL + slot)); // and goes to the forwarder
       }
-      // Slice of M_t to the CTA that owns frame t, for its read-out.
-      const int dst = t % P;
-      const int jo = t / P;
-      const int u = jo & 1;
-      if (!warp_wait(bar(L::B_MO_EMPTY + 2 * dst + u), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty)) {
-        ok = false;
-        break;
-      }
-      if (act) {
-        const uint32_t base = mapa(mo_buf(u) + rank * (kD * L::RW), dst);
-#pragma unroll
-        for (int c = 0; c < NC / 8; ++c) {
-          uint4 h, l;
-          split8(&m[8 * c], h, l);
-          const uint32_t off = swz_off(row, c, L::RW, L::SWZ_BITS);
-          st_cluster_v4(base + off, h);
-          st_cluster_v4(base + L::MO_PART + off, l);
-        }
-      }
-      fence_proxy_async_cluster();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
     }
     if (ok && act && p.state_out) {
 #pragma unroll
@@ -606,10 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       }
     }
   } else if (warp >= 12) {
-    // ------------------------------------------------ output tiles: TMEM -> bf16 -> TMA store
+    // ------------------------------------------------ output tiles: TMEM -> bf16 -> global
     const int qd = warp & 3;
-    const int lrow = qd * 32 + lane;
-    const bool leader = (warp == 12 && lane == 0);
+    const int lrow = qd * 32 + lane;           // tile row = TMEM lane
     int n = 0;
     bool ok = true;
     for (int j = 0; j < nown && ok; ++j) {
@@ -633,36 +646,25 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_O_FREE + ob));
-        const int slot = n % L::NQ;                  // the Q tile this output came from
-        const uint32_t tile = q_slot(slot);
+        // All MMAs reading this frame's state are done: its buffer may be refilled.
+        if (i == ntile - 1 && warp == 12 && lane == 0)
+          for (int q = 0; q < P; ++q)
+            mbar_arrive_cluster(mapa(bar(L::B_MO_EMPTY + 2 * rank + (j & 1)), q));
+        const int grow = i * kTile + lrow;
+        if (grow < p.S) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)bh * T + f) * p.S + grow) * kD);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-          w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-          w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-          w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-          st_shared_v4(tile + swz_off(lrow, c, 128, 3), w);
-        }
-        fence_proxy_async_cta();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_STAGE + (n & 1)));
-        if (leader) {
-          if (!wait_bar(bar(L::B_STAGE + (n & 1)), (n >> 1) & 1, ctl, kStOut)) {
-            ok = false;
-            break;
+          for (int c = 0; c < 8; ++c) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+            dst[c] = w;
           }
-          tma_store_3d(&p.tm_o, tile, 0, i * kTile, bh * T + f);
-          bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(bar(L::B_Q_EMPTY + slot));
-          if (i == ntile - 1)
-            for (int q = 0; q < P; ++q)
-              mbar_arrive_cluster(mapa(bar(L::B_MO_EMPTY + 2 * rank + (j & 1)), q));
         }
       }
     }
-    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
@@ -787,6 +789,7 @@ cudaError_t launch_p(const Problem& pr) {
   p.beta = pr.beta;
   p.state_in = pr.state_in;
   p.state_out = pr.state_out;
+  p.out = static_cast<uint16_t*>(pr.out);
   p.status = status;
   p.T = pr.T;
   p.S = pr.S;
