@@ -39,15 +39,22 @@ def needs_build() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(debug: bool = False, verbose: bool = False, force: bool = False) -> str:
-    if not force and not debug and not needs_build():
+def build(debug: bool = False, verbose: bool = False, force: bool = False,
+          trace_out: str | None = None) -> str:
+    """Builds libgdn.so. With trace_out, builds instead a pipeline-trace variant
+    (GDN_TRACE: per-frame event timestamps of head 0, read with gdn_trace_copy)
+    at that path; the library the binding loads is left untouched."""
+    out = trace_out or LIB
+    if not force and not debug and not trace_out and not needs_build():
         return LIB
     cmd = [nvcc(), *ARCH, "-std=c++17", "-O3", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB, *sources(), "-lcudart_static", "-ldl", "-lrt",
+           "-I", INCLUDE, "-I", CSRC, "-o", out, *sources(), "-lcudart_static", "-ldl", "-lrt",
            "-lpthread"]
     if debug:
         cmd.insert(1, "-DGDN_DEBUG=1")
+    if trace_out:
+        cmd.insert(1, "-DGDN_TRACE=1")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,9 +63,11 @@ def build(debug: bool = False, verbose: bool = False, force: bool = False) -> st
         raise RuntimeError("nvcc failed building libgdn.so")
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    build(debug="--debug" in sys.argv, verbose="-v" in sys.argv, force=True)
-    print(LIB)
+    trace = None
+    if "--trace-out" in sys.argv:
+        trace = sys.argv[sys.argv.index("--trace-out") + 1]
+    print(build(debug="--debug" in sys.argv, verbose="-v" in sys.argv, force=True, trace_out=trace))

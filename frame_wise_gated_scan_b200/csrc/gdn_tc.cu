@@ -41,6 +41,22 @@ namespace gdn {
 
 __device__ unsigned int g_tc_status = 0;
 
+#ifdef GDN_TRACE
+// Event timeline of head 0's cluster (globaltimer ns), for pipeline analysis
+// builds only: [rank][event][frame or own-frame index].
+constexpr int kTraceRanks = 4, kTraceEvents = 16, kTraceFrames = 1024;
+__device__ unsigned long long g_trace[kTraceRanks * kTraceEvents * kTraceFrames];
+#define GDN_TRACE_EV(ev, idx)                                                              \
+  do {                                                                                     \
+    if (bh == 0 && (idx) < kTraceFrames)                                                   \
+      g_trace[((int)rank * kTraceEvents + (ev)) * kTraceFrames + (idx)] = globaltimer_ns(); \
+  } while (0)
+#else
+#define GDN_TRACE_EV(ev, idx) \
+  do {                        \
+  } while (0)
+#endif
+
 namespace {
 
 using namespace ptx;
@@ -62,13 +78,14 @@ enum : uint32_t {
 template <int P>
 struct Layout {
   static constexpr int NC = kD / P;                  // state columns per CTA
-  static constexpr int NAC = P == 4 ? 3 : 2;         // transition-operand slots
+  static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr int NKV = 2;                      // K/V tile pairs in flight
-  static constexpr int NQ = P == 1 ? 2 : 3;          // Q tiles in flight
+  static constexpr int NQ = P == 4 ? 3 : 2;          // Q tiles in flight
   static constexpr int NMS = P == 1 ? 2 : 4;         // state-slice ring (MMA operand + outbox)
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
-  static constexpr uint32_t C_BYTES = kD * NC * 4;                  // c slice, fp32 [64][NC]
+  static constexpr uint32_t C_BLK = kD * NC * 4;                    // c block, fp32 [64][NC]
+  static constexpr uint32_t C_BYTES = P * C_BLK;                    // c, by column block
   static constexpr uint32_t AC_SLOT = align1k(2 * AP_BYTES + C_BYTES);
   static constexpr uint32_t RW = NC * 2;                            // bytes per slice row
   static constexpr uint32_t SBO = 8 * RW;                           // 8-row group stride
@@ -103,7 +120,8 @@ struct Layout {
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_MS_FULL = B_DRAIN + 1;                     // [NMS] slice written
   static constexpr int B_MS_FREE = B_MS_FULL + NMS;                 // [NMS] slice forwarded
-  static constexpr int NBAR = B_MS_FREE + NMS;
+  static constexpr int B_E1_STAGED = B_MS_FREE + NMS;               // [2] A' and c staged locally
+  static constexpr int NBAR = B_E1_STAGED + 2;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -265,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_Q_EMPTY + i), 1);
     }
     for (int i = 0; i < NAC; ++i) {
-      mbar_init(bar(L::B_AC_FULL + i), 4);          // the producer's 4 epilogue warps
+      mbar_init(bar(L::B_AC_FULL + i), 1);          // the producer's leader (+ copied bytes)
       mbar_init(bar(L::B_AC_EMPTY + i), P);         // the forwarder of every CTA
     }
     for (int i = 0; i < 2; ++i) {
@@ -280,6 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_MS_FULL + i), 4);
       mbar_init(bar(L::B_MS_FREE + i), 1);
     }
+    mbar_init(bar(L::B_E1_STAGED + 0), 4);
+    mbar_init(bar(L::B_E1_STAGED + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
     mbar_init(bar(L::B_DRAIN), 1);
@@ -316,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           break;
         }
         mbar_arrive_expect_tx(bar(L::B_KV_FULL + slot), 2 * kTileBytes);
+        if (i == 0) GDN_TRACE_EV(11, j);
+        if (i == ntile - 1) GDN_TRACE_EV(12, j);
         tma_load_3d(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kTile, bh * T + f);
         tma_load_3d(kv_slot(slot) + kTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0, i * kTile,
                     bh * T + f);
@@ -337,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           break;
         }
         mbar_arrive_expect_tx(bar(L::B_Q_FULL + slot), kTileBytes);
+        if (i == 0) GDN_TRACE_EV(13, j);
         tma_load_3d(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, i * kTile, bh * T + f);
       }
       if (!ok) break;
@@ -372,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           mma_bf16(dt, aL, bH, id_chain, 1u);
         }
         mma_commit(bar(L::B_CHAIN_DONE));
+        GDN_TRACE_EV(0, t);
         ++t;
         progressed = true;
       }
@@ -392,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           mma_commit(bar(L::B_KV_EMPTY + slot));
           if (gi == ntile - 1) {
             mma_commit(bar(L::B_GB_FULL + b));
+            GDN_TRACE_EV(14, gj);
             gi = 0;
             ++gj;
           } else {
@@ -423,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           }
           mma_commit(bar(L::B_Q_EMPTY + slot));
           mma_commit(bar(L::B_O_FULL + ob));
+          if (oi == 0) GDN_TRACE_EV(15, oj);
           ++qit;
           ++on;
           if (++oi == ntile) {
@@ -449,14 +475,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int t = 0; t < T; ++t) {
       const int slot = t % L::NMS;
       if (!warp_wait(bar(L::B_MS_FULL + slot), (t / L::NMS) & 1, ctl, kStChain)) break;
+      if (lane == 0) GDN_TRACE_EV(3, t);
       // The recurrence has read c_t and its MMA has read A'_t: release the slot.
-      if (lane == 0 && t + NAC < T)
+      if (lane == 0 && t + NAC < T) {
+        fence_proxy_async_cta();   // our reads of the slot precede the next bulk copy into it
         mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + t % NAC), (t + NAC) % P));
+      }
       const int dst = t % P;
       const int jo = t / P;
       const int u = jo & 1;
       if (!warp_wait(bar(L::B_MO_EMPTY + 2 * dst + u), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty))
         break;
+      if (lane == 0) GDN_TRACE_EV(4, t);
       const uint32_t src = ms_buf(slot);
       const uint32_t dhi = mapa(mo_buf(u) + rank * L::MS_PART, dst);
       for (uint32_t off = lane * 16; off < L::MS_PART; off += 512) {
@@ -468,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (lane == 0) {
         mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
         mbar_arrive(bar(L::B_MS_FREE + slot));
+        GDN_TRACE_EV(5, t);
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -497,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const float* gam = p.gamma + (size_t)bh * T;
     float g_next = __ldg(gam);
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
+    int t = 0;
+    for (; t < T; ++t) {
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
@@ -509,8 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         ok = false;
         break;
       }
+      if (lane == 0 && warp == 4) GDN_TRACE_EV(1, t);
       tc_fence_after();
-      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + (act ? row : 0) * NC * 4;
+      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + rank * L::C_BLK + (act ? row : 0) * NC * 4;
       const uint32_t mbuf = ms_buf(slot);
 #pragma unroll
       for (int c16 = 0; c16 < NC / 16; ++c16) {
@@ -543,11 +576,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (lane == 0) {
         mbar_arrive(bar(L::B_M_READY));        // M_t slice is the next MMA operand; TMEM free
         mbar_arrive(bar(L::B_MS_FULL + slot)); // and goes to the forwarder
+        if (warp == 4) GDN_TRACE_EV(2, t);
       }
     }
     if (ok && act && p.state_out) {
 #pragma unroll
       for (int jj = 0; jj < NC; ++jj) p.state_out[((size_t)bh * kD + row) * kD + j0 + jj] = m[jj];
+    }
+    if (!ok && warp == 4 && lane == 0) {
+      // Aborting: let bulk copies that peers may still have in flight into our
+      // transition slots land before this CTA can leave.
+      for (int tt = t; tt < T && tt < t + NAC; ++tt)
+        drain_bar(bar(L::B_AC_FULL + tt % NAC), (tt / NAC) & 1, ctl);
     }
   } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------ A' and c from [G; (K^T V)^T]
@@ -564,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const float g = __ldg(gam + f);
       const float be = __ldg(bet + f);
       if (!warp_wait(bar(L::B_GB_FULL + b), (j >> 1) & 1, ctl, kStProd)) break;
+      if (lane == 0 && warp == 8) GDN_TRACE_EV(6, j);
       tc_fence_after();
       uint32_t v[64];
 #pragma unroll
@@ -588,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int i = 0; i < NAC; ++i)
           if (i == s) waits[i] += 1;
       }
+      if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
       const uint32_t slot = ac_slot(s);
       if (lrow < kD) {
         // row lrow of A' = -gamma beta s^2 G, as bf16 hi + lo, K-major, 128-byte swizzle
@@ -600,24 +642,41 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           uint4 h, l;
           split8(x, h, l);
           const uint32_t off = swz_off(lrow, c, 128, 3);
-          for (int q = 0; q < P; ++q) {
-            st_cluster_v4(mapa(slot + off, q), h);
-            st_cluster_v4(mapa(slot + L::AP_BYTES + off, q), l);
-          }
+          st_shared_v4(slot + off, h);
+          st_shared_v4(slot + L::AP_BYTES + off, l);
         }
       } else {
-        // column (lrow - 64) of c = beta s K^T V, to the CTA that owns that state column
+        // column (lrow - 64) of c = beta s K^T V, into the block of the CTA owning that column
         const int jc = lrow - kD;
-        const uint32_t dst = mapa(slot + 2 * L::AP_BYTES + (jc % NC) * 4, jc / NC);
+        const uint32_t dst = slot + 2 * L::AP_BYTES + (jc / NC) * L::C_BLK + (jc % NC) * 4;
         const float coef = be * p.s;
 #pragma unroll
-        for (int i = 0; i < kD; ++i) st_cluster_f32(dst + i * NC * 4, coef * __uint_as_float(v[i]));
+        for (int i = 0; i < kD; ++i) {
+          const float cv = coef * __uint_as_float(v[i]);
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + i * NC * 4), "f"(cv) : "memory");
+        }
       }
-      fence_proxy_async_cluster();
+      fence_proxy_async_cta();     // visible to the bulk-copy engine
       __syncwarp();
-      if (lane == 0) {
-        for (int q = 0; q < P; ++q) mbar_arrive_cluster(mapa(bar(L::B_AC_FULL + s), q));
+      if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
+      uint32_t sent = 1;
+      if (warp == 8 && lane == 0) {
+        sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+        for (int q = 0; q < P && sent; ++q) {
+          if (q == (int)rank) {
+            mbar_arrive(bar(L::B_AC_FULL + s));
+          } else {
+            const uint32_t rbar = mapa(bar(L::B_AC_FULL + s), q);
+            const uint32_t cblk = 2 * L::AP_BYTES + q * L::C_BLK;
+            mbar_arrive_expect_tx_cluster(rbar, 2 * L::AP_BYTES + L::C_BLK);
+            bulk_copy_to_cluster(mapa(slot, q), slot, 2 * L::AP_BYTES, rbar);
+            bulk_copy_to_cluster(mapa(slot + cblk, q), slot + cblk, L::C_BLK, rbar);
+          }
+        }
+        GDN_TRACE_EV(8, j);
       }
+      sent = __shfl_sync(0xffffffffu, sent, 0);   // warp-uniform verdict (other warps: abort flag)
+      if (!sent) break;
     }
   } else if (warp >= 12) {
     // ------------------------------------------------ output tiles: TMEM -> bf16 -> global
@@ -633,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           ok = false;
           break;
         }
+        if (i == 0 && lane == 0 && warp == 12) GDN_TRACE_EV(9, j);
         tc_fence_after();
         uint32_t v[64];
 #pragma unroll
@@ -663,6 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             dst[c] = w;
           }
         }
+        if (i == ntile - 1 && lane == 0 && warp == 12) GDN_TRACE_EV(10, j);
       }
     }
   }
@@ -845,6 +906,13 @@ cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head) {
     default: return cudaErrorInvalidValue;
   }
 }
+
+#ifdef GDN_TRACE
+extern "C" __attribute__((visibility("default"))) int gdn_trace_copy(void* dst, size_t bytes) {
+  const size_t n = sizeof(g_trace) < bytes ? sizeof(g_trace) : bytes;
+  return cudaMemcpyFromSymbol(dst, g_trace, n) == cudaSuccess ? (int)n : -1;
+}
+#endif
 
 cudaError_t tc_read_status(unsigned int* status) {
   unsigned int zero = 0;
