@@ -44,7 +44,7 @@ __device__ unsigned int g_tc_status = 0;
 #ifdef GDN_TRACE
 // Event timeline of head 0's cluster (globaltimer ns), for pipeline analysis
 // builds only: [rank][event][frame or own-frame index].
-constexpr int kTraceRanks = 4, kTraceEvents = 16, kTraceFrames = 1024;
+constexpr int kTraceRanks = 4, kTraceEvents = 24, kTraceFrames = 1024;
 __device__ unsigned long long g_trace[kTraceRanks * kTraceEvents * kTraceFrames];
 #define GDN_TRACE_EV(ev, idx)                                                              \
   do {                                                                                     \
@@ -480,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (lane == 0 && t + NAC < T) {
         fence_proxy_async_cta();   // our reads of the slot precede the next bulk copy into it
         mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + t % NAC), (t + NAC) % P));
+        GDN_TRACE_EV(22, t);
       }
       const int dst = t % P;
       const int jo = t / P;
@@ -493,8 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         st_cluster_v4(dhi + off, ld_shared_u4(src + off));
         st_cluster_v4(dhi + L::MO_PART + off, ld_shared_u4(src + L::MS_PART + off));
       }
+      if (lane == 0) GDN_TRACE_EV(19, t);
       fence_proxy_async_cluster();
       __syncwarp();
+      if (lane == 0) GDN_TRACE_EV(20, t);
       if (lane == 0) {
         mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
         mbar_arrive(bar(L::B_MS_FREE + slot));
@@ -534,7 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
       const int slot = t % L::NMS;
-      if (!warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain) ||
+      const bool acok = warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain);
+      if (acok && lane == 0 && warp == 4) GDN_TRACE_EV(21, t);
+      if (!acok ||
           !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
           (t >= L::NMS &&
            !warp_wait(bar(L::B_MS_FREE + slot), ((t / L::NMS) & 1) ^ 1, ctl, kStChain))) {
@@ -656,12 +661,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + i * NC * 4), "f"(cv) : "memory");
         }
       }
+      if (lane == 0 && warp == 8) GDN_TRACE_EV(16, j);
       fence_proxy_async_cta();     // visible to the bulk-copy engine
       __syncwarp();
+      if (lane == 0 && warp == 8) GDN_TRACE_EV(17, j);
       if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
       uint32_t sent = 1;
       if (warp == 8 && lane == 0) {
         sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+        GDN_TRACE_EV(18, j);
         for (int q = 0; q < P && sent; ++q) {
           if (q == (int)rank) {
             mbar_arrive(bar(L::B_AC_FULL + s));
