@@ -77,50 +77,46 @@ enum : uint32_t {
 
 template <int P>
 struct Layout {
-  static constexpr int NC = kD / P;                  // state columns per CTA
-  static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr int NKV = 2;                      // K/V tile pairs in flight
-  static constexpr int NQ = P == 4 ? 3 : 2;          // Q tiles in flight
-  static constexpr int NMS = P == 1 ? 2 : 4;         // state-slice ring (MMA operand + outbox)
+  static constexpr int NQ = 2;                       // Q tiles in flight
+  static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
-  static constexpr uint32_t C_BLK = kD * NC * 4;                    // c block, fp32 [64][NC]
-  static constexpr uint32_t C_BYTES = P * C_BLK;                    // c, by column block
-  static constexpr uint32_t AC_SLOT = align1k(2 * AP_BYTES + C_BYTES);
-  static constexpr uint32_t RW = NC * 2;                            // bytes per slice row
-  static constexpr uint32_t SBO = 8 * RW;                           // 8-row group stride
-  static constexpr uint32_t MS_PART = kD * RW;                      // slice, hi or lo
-  static constexpr uint32_t MS_BUF = align1k(2 * MS_PART);
-  static constexpr uint32_t MO_PART = kD * kD * 2;                  // full M, hi or lo
-  static constexpr uint32_t MO_BUF = 2 * MO_PART;
-  static constexpr uint32_t SWZ_CODE = NC == 64 ? 2u : (NC == 32 ? 4u : 6u);
-  static constexpr int SWZ_BITS = NC == 64 ? 3 : (NC == 32 ? 2 : 1);
+  static constexpr uint32_t C_BYTES = kD * kD * 4;                  // c, fp32 row-major
+  static constexpr uint32_t AC_BYTES = 2 * AP_BYTES + C_BYTES;      // one bulk copy
+  static constexpr uint32_t AC_SLOT = align1k(AC_BYTES);
+  // State operand: bf16 hi then lo, each two MN-major blocks of 32 value
+  // columns (64-byte rows, 64-byte swizzle, 8-row groups of 512 bytes).
+  static constexpr uint32_t MB_RW = 64;
+  static constexpr uint32_t MB_SBO = 8 * MB_RW;
+  static constexpr uint32_t MB_BLOCK = kD * MB_RW;                  // 4 KB
+  static constexpr uint32_t M_PART = 2 * MB_BLOCK;                  // 8 KB
+  static constexpr uint32_t M_BUF = 2 * M_PART;                     // 16 KB
 
   static constexpr uint32_t OFF_KV = 0;
   static constexpr uint32_t OFF_Q = OFF_KV + NKV * KV_SLOT;
   static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
-  static constexpr uint32_t OFF_MS = OFF_AC + NAC * AC_SLOT;
-  static constexpr uint32_t OFF_MO = OFF_MS + NMS * MS_BUF;
-  static constexpr uint32_t OFF_BAR = OFF_MO + 2 * MO_BUF;
+  static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // recurrence operand
+  static constexpr uint32_t OFF_MO = OFF_MCH + M_BUF;               // 2 read-out operands
+  static constexpr uint32_t OFF_ACK = OFF_MO + 2 * M_BUF;           // 16 B per sender + source
+  static constexpr uint32_t OFF_BAR = OFF_ACK + 16 * (P + 1);
   // barrier indices (8 bytes each)
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_KV_EMPTY = B_KV_FULL + NKV;
   static constexpr int B_Q_FULL = B_KV_EMPTY + NKV;
   static constexpr int B_Q_EMPTY = B_Q_FULL + NQ;
-  static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;
-  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;
+  static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;      // [NAC] 1 arrival + copied bytes
+  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;    // [NAC] 1 arrival + 16 B per CTA
   static constexpr int B_GB_FULL = B_AC_EMPTY + NAC;
   static constexpr int B_GB_FREE = B_GB_FULL + 2;
   static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
   static constexpr int B_M_READY = B_CHAIN_DONE + 1;
   static constexpr int B_MO_FULL = B_M_READY + 1;
-  static constexpr int B_MO_EMPTY = B_MO_FULL + 2;                  // [P][2]
-  static constexpr int B_O_FULL = B_MO_EMPTY + 2 * P;
+  static constexpr int B_MO_EMPTY = B_MO_FULL + 2;
+  static constexpr int B_O_FULL = B_MO_EMPTY + 2;
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;
-  static constexpr int B_MS_FULL = B_DRAIN + 1;                     // [NMS] slice written
-  static constexpr int B_MS_FREE = B_MS_FULL + NMS;                 // [NMS] slice forwarded
-  static constexpr int B_E1_STAGED = B_MS_FREE + NMS;               // [2] A' and c staged locally
+  static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
   static constexpr int NBAR = B_E1_STAGED + 2;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
@@ -130,7 +126,8 @@ struct Layout {
   // TMEM columns (each region 128 lanes)
   static constexpr uint32_t T_GB = 0;        // 2 x 64: [G; (K^T V)^T] accumulators
   static constexpr uint32_t T_O = 128;       // 2 x 64: output tile accumulators
-  static constexpr uint32_t T_CHAIN = 256;   // NC columns, M = 64 layout
+  static constexpr uint32_t T_CHAIN = 256;   // 32 columns; value columns 0-31 in lanes
+                                             // 32q+0..15, columns 32-63 in lanes 32q+16..31
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -142,7 +139,6 @@ struct TcParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_o;
   const float* gamma;
   const float* beta;
   const float* state_in;
@@ -251,7 +247,6 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const C
 template <int P>
 __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<P>;
-  constexpr int NC = L::NC;
   constexpr int NAC = L::NAC;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -268,8 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   auto kv_slot = [&](int i) -> uint32_t { return sb + L::OFF_KV + i * L::KV_SLOT; };
   auto q_slot = [&](int i) -> uint32_t { return sb + L::OFF_Q + i * kTileBytes; };
   auto ac_slot = [&](int i) -> uint32_t { return sb + L::OFF_AC + i * L::AC_SLOT; };
-  auto ms_buf = [&](int i) -> uint32_t { return sb + L::OFF_MS + i * L::MS_BUF; };
-  auto mo_buf = [&](int i) -> uint32_t { return sb + L::OFF_MO + i * L::MO_BUF; };
+  auto mo_buf = [&](int i) -> uint32_t { return sb + L::OFF_MO + i * L::M_BUF; };
+  const uint32_t mch = sb + L::OFF_MCH;
+  const uint32_t ack_src = sb + L::OFF_ACK + 16u * P;
   const uint32_t tmem_ptr = sb + L::OFF_TMEM_PTR;
   Ctl ctl{sb + L::OFF_ABORT, p.status, P};
 
@@ -283,34 +279,31 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_Q_EMPTY + i), 1);
     }
     for (int i = 0; i < NAC; ++i) {
-      mbar_init(bar(L::B_AC_FULL + i), 1);          // the producer's leader (+ copied bytes)
-      mbar_init(bar(L::B_AC_EMPTY + i), P);         // the forwarder of every CTA
+      mbar_init(bar(L::B_AC_FULL + i), 1);
+      mbar_init(bar(L::B_AC_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
       mbar_init(bar(L::B_GB_FREE + i), 4);
-      mbar_init(bar(L::B_MO_FULL + i), P);          // the forwarder of every CTA
+      mbar_init(bar(L::B_MO_FULL + i), 4);
+      mbar_init(bar(L::B_MO_EMPTY + i), 1);
       mbar_init(bar(L::B_O_FULL + i), 1);
       mbar_init(bar(L::B_O_FREE + i), 4);
+      mbar_init(bar(L::B_E1_STAGED + i), 4);
     }
-    for (int i = 0; i < 2 * P; ++i) mbar_init(bar(L::B_MO_EMPTY + i), 1);
-    for (int i = 0; i < L::NMS; ++i) {
-      mbar_init(bar(L::B_MS_FULL + i), 4);
-      mbar_init(bar(L::B_MS_FREE + i), 1);
-    }
-    mbar_init(bar(L::B_E1_STAGED + 0), 4);
-    mbar_init(bar(L::B_E1_STAGED + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
     mbar_init(bar(L::B_DRAIN), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
+    // The first transition operands that other CTAs produce arrive by bulk copy.
+    for (int f = 0; f < NAC && f < T; ++f)
+      if (f % P != (int)rank) mbar_arrive_expect_tx(bar(L::B_AC_FULL + f), L::AC_BYTES);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
-    prefetch_tmap(&p.tm_o);
   }
   if (warp == 2) {
     tmem_alloc(tmem_ptr, L::TMEM_COLS);
@@ -319,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();   // every CTA's barriers exist before any remote arrive
+  cluster_sync();   // every CTA's barriers exist before any remote operation
   uint32_t tmem;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_ptr) : "memory");
 
@@ -368,31 +361,50 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
   } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------ MMA issuer
-    constexpr uint32_t id_chain = idesc_bf16(64, NC, 0, 1);    // A' K-major, M slice MN-major
+    constexpr uint32_t id_chain = idesc_bf16(64, 32, 0, 1);    // A' K-major, M half MN-major
     constexpr uint32_t id_gb = idesc_bf16(128, 64, 1, 1);      // [K V]^T and K, both MN-major
     constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);       // Q K-major, M MN-major
     int t = 0;                         // next frame of the recurrence
     int gj = 0, gi = 0, kvit = 0;      // [G; b^T] stream: own frame, tile, ring counter
     int oj = 0, oi = 0, qit = 0, on = 0;
+    int rel = 0;                       // next frame whose transition slot is to be released
     uint64_t t0 = globaltimer_ns();
     while (t < T || gj < nown || oj < nown) {
       bool progressed = false;
-      if (t < T && mbar_test(bar(L::B_M_READY), t & 1) &&
+      // Frame t-1 is fully consumed once the recurrence warps finished it (its MMA
+      // completed and they read its c): hand its slot to the producer of frame
+      // t-1+NAC right away.
+      if (rel < t && t < T && mbar_test(bar(L::B_M_READY), t & 1)) {
+        const int g = rel + NAC;
+        if (g < T) {
+          const int prod = g % P;
+          const int s = rel % NAC;
+          if (prod != (int)rank) mbar_arrive_expect_tx(bar(L::B_AC_FULL + s), L::AC_BYTES);
+          fence_proxy_async_cta();
+          bulk_copy_to_cluster(mapa(sb + L::OFF_ACK + 16u * rank, prod), ack_src, 16,
+                               mapa(bar(L::B_AC_EMPTY + s), prod));
+        }
+        ++rel;
+        progressed = true;
+      }
+      if (t < T && rel == t && mbar_test(bar(L::B_M_READY), t & 1) &&
           mbar_test(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1)) {
         tc_fence_after();
         const uint32_t ac = ac_slot(t % NAC);
-        const uint32_t mb = ms_buf((t + L::NMS - 1) % L::NMS);   // slice of M_{t-1}
-        const uint32_t dt = tmem + L::T_CHAIN;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
-          const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
-          const uint64_t bH = smem_desc(mb + kk * 2 * L::SBO, L::MS_PART, L::SBO, L::SWZ_CODE);
-          const uint64_t bL = smem_desc(mb + L::MS_PART + kk * 2 * L::SBO, L::MS_PART, L::SBO,
-                                        L::SWZ_CODE);
-          mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
-          mma_bf16(dt, aH, bL, id_chain, 1u);
-          mma_bf16(dt, aL, bH, id_chain, 1u);
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
+            const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
+            const uint32_t mb = mch + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
+            const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
+            const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
+            mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
+            mma_bf16(dt, aH, bL, id_chain, 1u);
+            mma_bf16(dt, aL, bH, id_chain, 1u);
+          }
         }
         mma_commit(bar(L::B_CHAIN_DONE));
         GDN_TRACE_EV(0, t);
@@ -440,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t a = smem_desc(qt + kk * 32, 16, 1024, 2);
-            const uint64_t bH = smem_desc(mo + kk * 2 * L::SBO, kD * L::RW, L::SBO, L::SWZ_CODE);
-            const uint64_t bL = smem_desc(mo + L::MO_PART + kk * 2 * L::SBO, kD * L::RW, L::SBO,
-                                          L::SWZ_CODE);
+            const uint64_t bH = smem_desc(mo + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
+            const uint64_t bL =
+                smem_desc(mo + L::M_PART + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
             mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
             mma_bf16(dO, a, bL, id_o, 1u);
           }
@@ -470,61 +482,29 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     mma_commit(bar(L::B_DRAIN));
     drain_bar(bar(L::B_DRAIN), 0, ctl);
-  } else if (warp == 3) {
-    // ------------------------------------------------ forwarder: state slices to frame owners
-    for (int t = 0; t < T; ++t) {
-      const int slot = t % L::NMS;
-      if (!warp_wait(bar(L::B_MS_FULL + slot), (t / L::NMS) & 1, ctl, kStChain)) break;
-      if (lane == 0) GDN_TRACE_EV(3, t);
-      // The recurrence has read c_t and its MMA has read A'_t: release the slot.
-      if (lane == 0 && t + NAC < T) {
-        fence_proxy_async_cta();   // our reads of the slot precede the next bulk copy into it
-        mbar_arrive_cluster(mapa(bar(L::B_AC_EMPTY + t % NAC), (t + NAC) % P));
-        GDN_TRACE_EV(22, t);
-      }
-      const int dst = t % P;
-      const int jo = t / P;
-      const int u = jo & 1;
-      if (!warp_wait(bar(L::B_MO_EMPTY + 2 * dst + u), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty))
-        break;
-      if (lane == 0) GDN_TRACE_EV(4, t);
-      const uint32_t src = ms_buf(slot);
-      const uint32_t dhi = mapa(mo_buf(u) + rank * L::MS_PART, dst);
-      for (uint32_t off = lane * 16; off < L::MS_PART; off += 512) {
-        st_cluster_v4(dhi + off, ld_shared_u4(src + off));
-        st_cluster_v4(dhi + L::MO_PART + off, ld_shared_u4(src + L::MS_PART + off));
-      }
-      if (lane == 0) GDN_TRACE_EV(19, t);
-      fence_proxy_async_cluster();
-      __syncwarp();
-      if (lane == 0) GDN_TRACE_EV(20, t);
-      if (lane == 0) {
-        mbar_arrive_cluster(mapa(bar(L::B_MO_FULL + u), dst));
-        mbar_arrive(bar(L::B_MS_FREE + slot));
-        GDN_TRACE_EV(5, t);
-      }
-    }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------ recurrence epilogue
+    // The accumulator holds A' M for the 64 state rows: value columns 0-31 of
+    // row 16q+i in TMEM lane 32q+i, columns 32-63 in lane 32q+16+i. So lane l
+    // of warp quarter q owns row 16q+(l%16), columns 32*(l/16)..+32.
     const int qd = warp & 3;
-    const int row = qd * 16 + lane;            // M = 64 accumulator: rows 16qd.. in lanes 32qd..
-    const bool act = lane < 16;
-    const int j0 = (int)rank * NC;
-    float m[NC];                               // fp32 state, row `row`, columns j0..j0+NC
+    const int hf = lane >> 4;
+    const int row = qd * 16 + (lane & 15);
+    float m[32];                               // fp32 state, row `row`, columns 32hf..32hf+31
 #pragma unroll
-    for (int jj = 0; jj < NC; ++jj)
-      m[jj] = (act && p.state_in) ? p.state_in[((size_t)bh * kD + row) * kD + j0 + jj] : 0.f;
-    if (act) {
-      const uint32_t b0 = ms_buf(L::NMS - 1);  // M_{-1} = M_0, read by the first MMA
+    for (int jj = 0; jj < 32; ++jj)
+      m[jj] = p.state_in ? p.state_in[((size_t)bh * kD + row) * kD + 32 * hf + jj] : 0.f;
+    auto store_state = [&](uint32_t buf) {
 #pragma unroll
-      for (int c = 0; c < NC / 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint4 h, l;
         split8(&m[8 * c], h, l);
-        const uint32_t off = swz_off(row, c, L::RW, L::SWZ_BITS);
-        st_shared_v4(b0 + off, h);
-        st_shared_v4(b0 + L::MS_PART + off, l);
+        const uint32_t off = hf * L::MB_BLOCK + swz_off(row, c, L::MB_RW, 2);
+        st_shared_v4(buf + off, h);
+        st_shared_v4(buf + L::M_PART + off, l);
       }
-    }
+    };
+    store_state(mch);                          // M_{-1} = M_0, read by the first MMA
     fence_proxy_async_cta();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::B_M_READY));
@@ -536,57 +516,54 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
-      const int slot = t % L::NMS;
+      const bool own = (t % P) == (int)rank;
+      const int jo = t / P;
       const bool acok = warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain);
       if (acok && lane == 0 && warp == 4) GDN_TRACE_EV(21, t);
-      if (!acok ||
-          !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
-          (t >= L::NMS &&
-           !warp_wait(bar(L::B_MS_FREE + slot), ((t / L::NMS) & 1) ^ 1, ctl, kStChain))) {
+      if (!acok || !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
+          (own && !warp_wait(bar(L::B_MO_EMPTY + (jo & 1)), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty))) {
         ok = false;
         break;
       }
       if (lane == 0 && warp == 4) GDN_TRACE_EV(1, t);
       tc_fence_after();
-      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + rank * L::C_BLK + (act ? row : 0) * NC * 4;
-      const uint32_t mbuf = ms_buf(slot);
-#pragma unroll
-      for (int c16 = 0; c16 < NC / 16; ++c16) {
-        uint32_t d[16];
-        tmem_ld16(tmem + L::T_CHAIN + 16 * c16 + ((uint32_t)(qd * 32) << 16), d);
+      uint32_t d[32];
+      {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tmem + L::T_CHAIN + ((uint32_t)(qd * 32) << 16), r0);
+        tmem_ld16(tmem + L::T_CHAIN + 16 + ((uint32_t)(qd * 32) << 16), r1);
         tmem_wait_ld();
-        if (act) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const float4 cv = ld_shared_f4(crow + 64 * c16 + 16 * c4);
-            float* mm = &m[16 * c16 + 4 * c4];
-            mm[0] = fmaf(g, mm[0], __uint_as_float(d[4 * c4 + 0])) + cv.x;
-            mm[1] = fmaf(g, mm[1], __uint_as_float(d[4 * c4 + 1])) + cv.y;
-            mm[2] = fmaf(g, mm[2], __uint_as_float(d[4 * c4 + 2])) + cv.z;
-            mm[3] = fmaf(g, mm[3], __uint_as_float(d[4 * c4 + 3])) + cv.w;
-          }
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            uint4 h, l;
-            split8(&m[16 * c16 + 8 * h8], h, l);
-            const uint32_t off = swz_off(row, 2 * c16 + h8, L::RW, L::SWZ_BITS);
-            st_shared_v4(mbuf + off, h);
-            st_shared_v4(mbuf + L::MS_PART + off, l);
-          }
+        for (int e = 0; e < 16; ++e) {
+          d[e] = r0[e];
+          d[16 + e] = r1[e];
         }
       }
+      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + (row * kD + 32 * hf) * 4;
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 cv = ld_shared_f4(crow + 16 * c4);
+        float* mm = &m[4 * c4];
+        mm[0] = fmaf(g, mm[0], __uint_as_float(d[4 * c4 + 0])) + cv.x;
+        mm[1] = fmaf(g, mm[1], __uint_as_float(d[4 * c4 + 1])) + cv.y;
+        mm[2] = fmaf(g, mm[2], __uint_as_float(d[4 * c4 + 2])) + cv.z;
+        mm[3] = fmaf(g, mm[3], __uint_as_float(d[4 * c4 + 3])) + cv.w;
+      }
+      store_state(mch);
+      if (own) store_state(mo_buf(jo & 1));
       tc_fence_before();
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(L::B_M_READY));        // M_t slice is the next MMA operand; TMEM free
-        mbar_arrive(bar(L::B_MS_FULL + slot)); // and goes to the forwarder
+        mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
+        if (own) mbar_arrive(bar(L::B_MO_FULL + (jo & 1)));
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
     }
-    if (ok && act && p.state_out) {
+    if (ok && p.state_out) {
 #pragma unroll
-      for (int jj = 0; jj < NC; ++jj) p.state_out[((size_t)bh * kD + row) * kD + j0 + jj] = m[jj];
+      for (int jj = 0; jj < 32; ++jj)
+        p.state_out[((size_t)bh * kD + row) * kD + 32 * hf + jj] = m[jj];
     }
     if (!ok && warp == 4 && lane == 0) {
       // Aborting: let bulk copies that peers may still have in flight into our
@@ -623,8 +600,30 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_GB_FREE + b));
+      // Convert first, then wait for the slot: after the wait only stores remain.
+      // A' rows are packed in place: chunk c (8 values) becomes its 4 hi words
+      // in v[8c..8c+3] and its 4 lo words in v[8c+4..8c+7].
+      if (lrow < kD) {
+        const float coef = -g * be * p.s2;       // A' = -gamma beta s^2 G
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = coef * __uint_as_float(v[8 * c + e]);
+          uint4 h, l;
+          split8(x, h, l);
+          v[8 * c + 0] = h.x; v[8 * c + 1] = h.y; v[8 * c + 2] = h.z; v[8 * c + 3] = h.w;
+          v[8 * c + 4] = l.x; v[8 * c + 5] = l.y; v[8 * c + 6] = l.z; v[8 * c + 7] = l.w;
+        }
+      } else {
+        const float coef = be * p.s;             // c = beta s K^T V
+#pragma unroll
+        for (int i = 0; i < kD; ++i) v[i] = __float_as_uint(coef * __uint_as_float(v[i]));
+      }
       const int s = f % NAC;
       if (f >= NAC) {
+        // The slot is free once every CTA's 16-byte release copy has landed.
+        if (warp == 8 && lane == 0) mbar_arrive_expect_tx(bar(L::B_AC_EMPTY + s), 16u * P);
         int w = 0;
 #pragma unroll
         for (int i = 0; i < NAC; ++i)
@@ -637,49 +636,32 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
       const uint32_t slot = ac_slot(s);
       if (lrow < kD) {
-        // row lrow of A' = -gamma beta s^2 G, as bf16 hi + lo, K-major, 128-byte swizzle
-        const float coef = -g * be * p.s2;
+        // row lrow of A', bf16 hi + lo, K-major, 128-byte swizzle
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = coef * __uint_as_float(v[8 * c + e]);
-          uint4 h, l;
-          split8(x, h, l);
           const uint32_t off = swz_off(lrow, c, 128, 3);
-          st_shared_v4(slot + off, h);
-          st_shared_v4(slot + L::AP_BYTES + off, l);
+          st_shared_v4(slot + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]));
+          st_shared_v4(slot + L::AP_BYTES + off,
+                       make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]));
         }
       } else {
-        // column (lrow - 64) of c = beta s K^T V, into the block of the CTA owning that column
-        const int jc = lrow - kD;
-        const uint32_t dst = slot + 2 * L::AP_BYTES + (jc / NC) * L::C_BLK + (jc % NC) * 4;
-        const float coef = be * p.s;
+        // column (lrow - 64) of c, fp32 row-major
+        const uint32_t dst = slot + 2 * L::AP_BYTES + (lrow - kD) * 4;
 #pragma unroll
-        for (int i = 0; i < kD; ++i) {
-          const float cv = coef * __uint_as_float(v[i]);
-          asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + i * NC * 4), "f"(cv) : "memory");
-        }
+        for (int i = 0; i < kD; ++i)
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + i * kD * 4), "r"(v[i]) : "memory");
       }
-      if (lane == 0 && warp == 8) GDN_TRACE_EV(16, j);
-      fence_proxy_async_cta();     // visible to the bulk-copy engine
+      fence_proxy_async_cta();     // visible to the MMA and to the bulk-copy engine
       __syncwarp();
-      if (lane == 0 && warp == 8) GDN_TRACE_EV(17, j);
       if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
       uint32_t sent = 1;
       if (warp == 8 && lane == 0) {
         sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
-        GDN_TRACE_EV(18, j);
-        for (int q = 0; q < P && sent; ++q) {
-          if (q == (int)rank) {
-            mbar_arrive(bar(L::B_AC_FULL + s));
-          } else {
-            const uint32_t rbar = mapa(bar(L::B_AC_FULL + s), q);
-            const uint32_t cblk = 2 * L::AP_BYTES + q * L::C_BLK;
-            mbar_arrive_expect_tx_cluster(rbar, 2 * L::AP_BYTES + L::C_BLK);
-            bulk_copy_to_cluster(mapa(slot, q), slot, 2 * L::AP_BYTES, rbar);
-            bulk_copy_to_cluster(mapa(slot + cblk, q), slot + cblk, L::C_BLK, rbar);
-          }
+        if (sent) {
+          mbar_arrive(bar(L::B_AC_FULL + s));
+          for (int q = 0; q < P; ++q)
+            if (q != (int)rank)
+              bulk_copy_to_cluster(mapa(slot, q), slot, L::AC_BYTES, mapa(bar(L::B_AC_FULL + s), q));
         }
         GDN_TRACE_EV(8, j);
       }
@@ -715,9 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_O_FREE + ob));
         // All MMAs reading this frame's state are done: its buffer may be refilled.
-        if (i == ntile - 1 && warp == 12 && lane == 0)
-          for (int q = 0; q < P; ++q)
-            mbar_arrive_cluster(mapa(bar(L::B_MO_EMPTY + 2 * rank + (j & 1)), q));
+        if (i == ntile - 1 && warp == 12 && lane == 0) mbar_arrive(bar(L::B_MO_EMPTY + (j & 1)));
         const int grow = i * kTile + lrow;
         if (grow < p.S) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)bh * T + f) * p.S + grow) * kD);
@@ -850,7 +830,7 @@ cudaError_t launch_p(const Problem& pr) {
   TcParams p;
   const long long frames = (long long)pr.B * pr.H * pr.T;
   if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames) ||
-      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames))
+      !make_map(&p.tm_v, pr.v, pr.S, frames))
     return cudaErrorInvalidValue;
   unsigned int* status = status_word();
   if (!status) return cudaErrorInvalidDevice;
