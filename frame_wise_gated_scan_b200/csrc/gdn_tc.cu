@@ -67,12 +67,13 @@ constexpr int kD = 64;
 constexpr int kTile = 128;                                      // rows per tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;                 // 16 KB
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+constexpr int kRing = 8;                                        // frames per head in the ring
 
 // Status codes recorded in g_tc_status (bit per waiting role).
 enum : uint32_t {
   kStKvLoad = 1u << 0, kStQLoad = 1u << 1, kStMma = 1u << 2, kStChain = 1u << 3,
   kStProd = 1u << 4, kStOut = 1u << 5, kStDrain = 1u << 6, kStMoEmpty = 1u << 7,
-  kStAcEmpty = 1u << 8
+  kStAcEmpty = 1u << 8, kStRing = 1u << 9
 };
 
 template <int P>
@@ -98,15 +99,14 @@ struct Layout {
   static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
   static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // recurrence operand
   static constexpr uint32_t OFF_MO = OFF_MCH + M_BUF;               // 2 read-out operands
-  static constexpr uint32_t OFF_ACK = OFF_MO + 2 * M_BUF;           // 16 B per sender + source
-  static constexpr uint32_t OFF_BAR = OFF_ACK + 16 * (P + 1);
+  static constexpr uint32_t OFF_BAR = OFF_MO + 2 * M_BUF;
   // barrier indices (8 bytes each)
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_KV_EMPTY = B_KV_FULL + NKV;
   static constexpr int B_Q_FULL = B_KV_EMPTY + NKV;
   static constexpr int B_Q_EMPTY = B_Q_FULL + NQ;
-  static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;      // [NAC] 1 arrival + copied bytes
-  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;    // [NAC] 1 arrival + 16 B per CTA
+  static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;      // [NAC] operands of the frame ready
+  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;    // [NAC] frame consumed locally
   static constexpr int B_GB_FULL = B_AC_EMPTY + NAC;
   static constexpr int B_GB_FREE = B_GB_FULL + 2;
   static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
@@ -117,7 +117,8 @@ struct Layout {
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
-  static constexpr int NBAR = B_E1_STAGED + 2;
+  static constexpr int B_LD_DONE = B_E1_STAGED + 2;     // [NAC] loader's bulk load landed
+  static constexpr int NBAR = B_LD_DONE + NAC;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -145,6 +146,11 @@ struct TcParams {
   float* state_out;
   uint16_t* out;           // bf16 bit patterns
   unsigned int* status;
+  // Transition operands shared by the CTAs of a head (P > 1), per head:
+  // kRing frames of [A' hi | A' lo | c], their ready flags and per-CTA progress.
+  uint8_t* ring;                     // [heads][kRing][AC_BYTES]
+  unsigned long long* ring_flag;     // [heads][kRing]: frame + 1 once published
+  unsigned long long* ring_loaded;   // [heads][P]: frames loaded by each CTA
   int T;
   int S;
   int ntile;
@@ -244,6 +250,22 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const C
   }
 }
 
+// Bounded poll of a global counter written by another CTA (acquire).
+__device__ __forceinline__ bool wait_global_ge(const unsigned long long* ptr,
+                                               unsigned long long v, const Ctl& c,
+                                               uint32_t code) {
+  if (ld_acquire_gpu_u64(ptr) >= v) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (ld_acquire_gpu_u64(ptr) >= v) return true;
+    if (aborted(c)) return false;
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      raise_abort(c, code);
+      return false;
+    }
+  }
+}
+
 template <int P>
 __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<P>;
@@ -265,7 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   auto ac_slot = [&](int i) -> uint32_t { return sb + L::OFF_AC + i * L::AC_SLOT; };
   auto mo_buf = [&](int i) -> uint32_t { return sb + L::OFF_MO + i * L::M_BUF; };
   const uint32_t mch = sb + L::OFF_MCH;
-  const uint32_t ack_src = sb + L::OFF_ACK + 16u * P;
   const uint32_t tmem_ptr = sb + L::OFF_TMEM_PTR;
   Ctl ctl{sb + L::OFF_ABORT, p.status, P};
 
@@ -281,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int i = 0; i < NAC; ++i) {
       mbar_init(bar(L::B_AC_FULL + i), 1);
       mbar_init(bar(L::B_AC_EMPTY + i), 1);
+      mbar_init(bar(L::B_LD_DONE + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
@@ -296,9 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mbar_init(bar(L::B_DRAIN), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
-    // The first transition operands that other CTAs produce arrive by bulk copy.
-    for (int f = 0; f < NAC && f < T; ++f)
-      if (f % P != (int)rank) mbar_arrive_expect_tx(bar(L::B_AC_FULL + f), L::AC_BYTES);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&p.tm_q);
@@ -312,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();   // every CTA's barriers exist before any remote operation
+  cluster_sync();   // the CTAs of a head start together
   uint32_t tmem;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_ptr) : "memory");
 
@@ -371,19 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     uint64_t t0 = globaltimer_ns();
     while (t < T || gj < nown || oj < nown) {
       bool progressed = false;
-      // Frame t-1 is fully consumed once the recurrence warps finished it (its MMA
-      // completed and they read its c): hand its slot to the producer of frame
-      // t-1+NAC right away.
+      // Frame t-1 is fully consumed once the recurrence warps finished it (its
+      // MMA completed and they read its c): its slot may be refilled.
       if (rel < t && t < T && mbar_test(bar(L::B_M_READY), t & 1)) {
-        const int g = rel + NAC;
-        if (g < T) {
-          const int prod = g % P;
-          const int s = rel % NAC;
-          if (prod != (int)rank) mbar_arrive_expect_tx(bar(L::B_AC_FULL + s), L::AC_BYTES);
-          fence_proxy_async_cta();
-          bulk_copy_to_cluster(mapa(sb + L::OFF_ACK + 16u * rank, prod), ack_src, 16,
-                               mapa(bar(L::B_AC_EMPTY + s), prod));
-        }
+        mbar_arrive(bar(L::B_AC_EMPTY + rel % NAC));
         ++rel;
         progressed = true;
       }
@@ -482,6 +492,34 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     mma_commit(bar(L::B_DRAIN));
     drain_bar(bar(L::B_DRAIN), 0, ctl);
+  } else if (warp == 3 && lane == 0 && P > 1) {
+    // ------------------------------------------------ loader of other CTAs' transition operands
+    int ldn[NAC];
+#pragma unroll
+    for (int i = 0; i < NAC; ++i) ldn[i] = 0;
+    for (int t = 0; t < T; ++t) {
+      const int s = t % NAC;
+      if (t % P != (int)rank) {
+        if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
+        const size_t rs = (size_t)bh * kRing + t % kRing;
+        if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
+        GDN_TRACE_EV(16, t);
+        fence_proxy_async_global();
+        int n = 0;
+#pragma unroll
+        for (int i = 0; i < NAC; ++i)
+          if (i == s) n = ldn[i]++;
+        mbar_arrive_expect_tx(bar(L::B_LD_DONE + s), L::AC_BYTES);
+        bulk_load_global(ac_slot(s), p.ring + rs * L::AC_BYTES, L::AC_BYTES, bar(L::B_LD_DONE + s));
+        // Wait for the bytes even when aborting: the copy targets this CTA.
+        drain_bar(bar(L::B_LD_DONE + s), n & 1, ctl);
+        mbar_arrive(bar(L::B_AC_FULL + s));
+        GDN_TRACE_EV(17, t);
+      }
+      // Frames up to t are loaded (or were this CTA's own): their ring slots may be reused.
+      st_release_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t + 1));
+      if (aborted(ctl)) break;
+    }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------ recurrence epilogue
     // The accumulator holds A' M for the 64 state rows: value columns 0-31 of
@@ -565,19 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       for (int jj = 0; jj < 32; ++jj)
         p.state_out[((size_t)bh * kD + row) * kD + 32 * hf + jj] = m[jj];
     }
-    if (!ok && warp == 4 && lane == 0) {
-      // Aborting: let bulk copies that peers may still have in flight into our
-      // transition slots land before this CTA can leave.
-      for (int tt = t; tt < T && tt < t + NAC; ++tt)
-        drain_bar(bar(L::B_AC_FULL + tt % NAC), (tt / NAC) & 1, ctl);
-    }
   } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------ A' and c from [G; (K^T V)^T]
     const int qd = warp & 3;
     const int lrow = qd * 32 + lane;           // accumulator row = TMEM lane
-    int waits[NAC];
-#pragma unroll
-    for (int i = 0; i < NAC; ++i) waits[i] = 0;
     const float* gam = p.gamma + (size_t)bh * T;
     const float* bet = p.beta + (size_t)bh * T;
     for (int j = 0; j < nown; ++j) {
@@ -621,18 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int i = 0; i < kD; ++i) v[i] = __float_as_uint(coef * __uint_as_float(v[i]));
       }
       const int s = f % NAC;
-      if (f >= NAC) {
-        // The slot is free once every CTA's 16-byte release copy has landed.
-        if (warp == 8 && lane == 0) mbar_arrive_expect_tx(bar(L::B_AC_EMPTY + s), 16u * P);
-        int w = 0;
-#pragma unroll
-        for (int i = 0; i < NAC; ++i)
-          if (i == s) w = waits[i];
-        if (!warp_wait(bar(L::B_AC_EMPTY + s), w & 1, ctl, kStAcEmpty)) break;
-#pragma unroll
-        for (int i = 0; i < NAC; ++i)
-          if (i == s) waits[i] += 1;
-      }
+      // The local slot is free once frame f - NAC has been consumed here.
+      if (!warp_wait(bar(L::B_AC_EMPTY + s), ((f / NAC) & 1) ^ 1, ctl, kStAcEmpty)) break;
       if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
       const uint32_t slot = ac_slot(s);
       if (lrow < kD) {
@@ -657,11 +676,26 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       uint32_t sent = 1;
       if (warp == 8 && lane == 0) {
         sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
-        if (sent) {
-          mbar_arrive(bar(L::B_AC_FULL + s));
-          for (int q = 0; q < P; ++q)
+        const size_t rs = (size_t)bh * kRing + f % kRing;
+        if (sent && P > 1) {
+          // Publish to the other CTAs of the head through the ring: its slot is
+          // free once each of them has loaded frame f - kRing.
+          for (int q = 0; q < P && sent && f >= kRing; ++q)
             if (q != (int)rank)
-              bulk_copy_to_cluster(mapa(slot, q), slot, L::AC_BYTES, mapa(bar(L::B_AC_FULL + s), q));
+              sent = wait_global_ge(p.ring_loaded + (size_t)bh * P + q,
+                                    (unsigned long long)(f - kRing + 1), ctl, kStRing);
+          if (sent) {
+            fence_proxy_async_global();
+            bulk_store_global(p.ring + rs * L::AC_BYTES, slot, L::AC_BYTES);
+            bulk_commit();
+            bulk_wait_read0();     // the local slot may be consumed and reused from here on
+          }
+        }
+        if (sent) mbar_arrive(bar(L::B_AC_FULL + s));
+        if (sent && P > 1) {
+          bulk_wait0();
+          fence_proxy_async_global();
+          st_release_gpu_u64(p.ring_flag + rs, (unsigned long long)(f + 1));
         }
         GDN_TRACE_EV(8, j);
       }
@@ -847,19 +881,40 @@ cudaError_t launch_p(const Problem& pr) {
   const double sd = 1.0 / ((double)kD * (double)pr.S);
   p.s2 = (float)sd;
 
+  // Ring of transition operands shared by the CTAs of each head (P > 1):
+  // stream-ordered scratch, released right after the launch on the same stream.
+  const size_t heads = (size_t)pr.B * pr.H;
+  const size_t ring_bytes = heads * kRing * Layout<P>::AC_BYTES;
+  const size_t ctrl_bytes = heads * (kRing + P) * sizeof(unsigned long long);
+  void* scratch = nullptr;
+  p.ring = nullptr;
+  p.ring_flag = nullptr;
+  p.ring_loaded = nullptr;
+  if (P > 1) {
+    e = cudaMallocAsync(&scratch, ring_bytes + ctrl_bytes, pr.stream);
+    if (e != cudaSuccess) return e;
+    p.ring = static_cast<uint8_t*>(scratch);
+    p.ring_flag = reinterpret_cast<unsigned long long*>(p.ring + ring_bytes);
+    p.ring_loaded = p.ring_flag + heads * kRing;
+    e = cudaMemsetAsync(p.ring_flag, 0, ctrl_bytes, pr.stream);
+    if (e != cudaSuccess) {
+      cudaFreeAsync(scratch, pr.stream);
+      return e;
+    }
+  }
+
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = P;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(pr.B * pr.H * P), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Layout<P>::SMEM_ALLOC;
-  cfg.stream = pr.stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<P>, p);
+  cfg.gridDim = dim3((unsigned)(pr.B * pr.H * P), 1, 1);  e = cudaLaunchKernelEx(&cfg, gdn_tc_kernel<P>, p);
+  if (scratch) {
+    const cudaError_t ef = cudaFreeAsync(scratch, pr.stream);
+    if (e == cudaSuccess) e = ef;
+  }
+  return e;
 }
 
 }  // namespace
