@@ -73,7 +73,7 @@ constexpr int kRing = 8;                                        // frames per he
 enum : uint32_t {
   kStKvLoad = 1u << 0, kStQLoad = 1u << 1, kStMma = 1u << 2, kStChain = 1u << 3,
   kStProd = 1u << 4, kStOut = 1u << 5, kStDrain = 1u << 6, kStMoEmpty = 1u << 7,
-  kStAcEmpty = 1u << 8, kStRing = 1u << 9
+  kStAcEmpty = 1u << 8, kStRing = 1u << 9, kStConfig = 1u << 10
 };
 
 template <int P>
@@ -271,6 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   using L = Layout<P>;
   constexpr int NAC = L::NAC;
   extern __shared__ uint8_t smem_raw[];
+  {
+    // A launch with the wrong block size or too little shared memory records
+    // an error and touches nothing (every thread of every CTA returns here).
+    uint32_t dsmem;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dsmem));
+    if (blockDim.x != kThreads || blockDim.y != 1 || blockDim.z != 1 || dsmem < L::SMEM_ALLOC) {
+      if (threadIdx.x == 0) atomicOr(p.status, kStConfig);
+      return;
+    }
+  }
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;         // 1 KB aligned base, same in every CTA
   const int warp = threadIdx.x >> 5;
@@ -909,7 +919,13 @@ cudaError_t launch_p(const Problem& pr) {
   attr[0].val.clusterDim.x = P;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(pr.B * pr.H * P), 1, 1);  e = cudaLaunchKernelEx(&cfg, gdn_tc_kernel<P>, p);
+  cfg.gridDim = dim3((unsigned)(pr.B * pr.H * P), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<P>::SMEM_ALLOC;
+  cfg.stream = pr.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gdn_tc_kernel<P>, p);
   if (scratch) {
     const cudaError_t ef = cudaFreeAsync(scratch, pr.stream);
     if (e == cudaSuccess) e = ef;
