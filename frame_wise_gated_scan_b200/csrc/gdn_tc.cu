@@ -118,7 +118,8 @@ struct Layout {
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
   static constexpr int B_LD_DONE = B_E1_STAGED + 2;     // [NAC] loader's bulk load landed
-  static constexpr int NBAR = B_LD_DONE + NAC;
+  static constexpr int B_OWN_FREE = B_LD_DONE + NAC;    // [NAC] slot free for an own frame
+  static constexpr int NBAR = B_OWN_FREE + NAC;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_AC_FULL + i), 1);
       mbar_init(bar(L::B_AC_EMPTY + i), 1);
       mbar_init(bar(L::B_LD_DONE + i), 1);
+      mbar_init(bar(L::B_OWN_FREE + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
@@ -507,10 +509,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     int ldn[NAC];
 #pragma unroll
     for (int i = 0; i < NAC; ++i) ldn[i] = 0;
+    // Slots are handed out strictly in frame order here, so every wait below is
+    // for the next phase of its barrier.
     for (int t = 0; t < T; ++t) {
       const int s = t % NAC;
-      if (t % P != (int)rank) {
-        if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
+      if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
+      if (t % P == (int)rank) {
+        mbar_arrive(bar(L::B_OWN_FREE + s));     // this CTA's producer fills it
+      } else {
         const size_t rs = (size_t)bh * kRing + t % kRing;
         if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
         GDN_TRACE_EV(16, t);
@@ -619,6 +625,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int lrow = qd * 32 + lane;           // accumulator row = TMEM lane
     const float* gam = p.gamma + (size_t)bh * T;
     const float* bet = p.beta + (size_t)bh * T;
+    int own_n[NAC];                              // own frames filled per slot so far
+#pragma unroll
+    for (int i = 0; i < NAC; ++i) own_n[i] = 0;
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
       const int b = j & 1;
@@ -660,8 +669,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int i = 0; i < kD; ++i) v[i] = __float_as_uint(coef * __uint_as_float(v[i]));
       }
       const int s = f % NAC;
-      // The local slot is free once frame f - NAC has been consumed here.
-      if (!warp_wait(bar(L::B_AC_EMPTY + s), ((f / NAC) & 1) ^ 1, ctl, kStAcEmpty)) break;
+      // The local slot is free once frame f - NAC has been consumed here. With one
+      // CTA per head every frame is ours and the release phases come in order;
+      // otherwise the loader hands the slot over in frame order.
+      bool slot_ok;
+      if (P == 1) {
+        slot_ok = warp_wait(bar(L::B_AC_EMPTY + s), ((f / NAC) & 1) ^ 1, ctl, kStAcEmpty);
+      } else {
+        int n = 0;
+#pragma unroll
+        for (int i = 0; i < NAC; ++i)
+          if (i == s) n = own_n[i]++;
+        slot_ok = warp_wait(bar(L::B_OWN_FREE + s), n & 1, ctl, kStAcEmpty);
+      }
+      if (!slot_ok) break;
       if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
       const uint32_t slot = ac_slot(s);
       if (lrow < kD) {
