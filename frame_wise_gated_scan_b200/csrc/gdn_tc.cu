@@ -83,7 +83,7 @@ struct Layout {
   static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
-  static constexpr uint32_t C_BYTES = kD * kD * 4;                  // c, fp32 row-major
+  static constexpr uint32_t C_BYTES = kD * kD * 4;                  // c^T, fp32: row j = column j of c
   static constexpr uint32_t AC_BYTES = 2 * AP_BYTES + C_BYTES;      // one bulk copy
   static constexpr uint32_t AC_SLOT = align1k(AC_BYTES);
   // State operand: bf16 hi then lo, each two MN-major blocks of 32 value
@@ -118,8 +118,7 @@ struct Layout {
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
   static constexpr int B_LD_DONE = B_E1_STAGED + 2;     // [NAC] loader's bulk load landed
-  static constexpr int B_OWN_FREE = B_LD_DONE + NAC;    // [NAC] slot free for an own frame
-  static constexpr int NBAR = B_OWN_FREE + NAC;
+  static constexpr int NBAR = B_LD_DONE + NAC;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -314,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_AC_FULL + i), 1);
       mbar_init(bar(L::B_AC_EMPTY + i), 1);
       mbar_init(bar(L::B_LD_DONE + i), 1);
-      mbar_init(bar(L::B_OWN_FREE + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
@@ -509,14 +507,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     int ldn[NAC];
 #pragma unroll
     for (int i = 0; i < NAC; ++i) ldn[i] = 0;
-    // Slots are handed out strictly in frame order here, so every wait below is
-    // for the next phase of its barrier.
+    // Every frame, this CTA's own included, arrives through the ring, in frame
+    // order, so each wait below is for the next phase of its barrier.
     for (int t = 0; t < T; ++t) {
       const int s = t % NAC;
       if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
-      if (t % P == (int)rank) {
-        mbar_arrive(bar(L::B_OWN_FREE + s));     // this CTA's producer fills it
-      } else {
+      {
         const size_t rs = (size_t)bh * kRing + t % kRing;
         if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
         GDN_TRACE_EV(16, t);
@@ -532,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         mbar_arrive(bar(L::B_AC_FULL + s));
         GDN_TRACE_EV(17, t);
       }
-      // Frames up to t are loaded (or were this CTA's own): their ring slots may be reused.
+      // Frames up to t are loaded here: their ring slots may be reused.
       st_release_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t + 1));
       if (aborted(ctl)) break;
     }
@@ -593,15 +589,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           d[16 + e] = r1[e];
         }
       }
-      const uint32_t crow = ac_slot(s) + 2 * L::AP_BYTES + (row * kD + 32 * hf) * 4;
+      // c[row][32hf + jj] = c^T[32hf + jj][row]
+      const uint32_t ccol = ac_slot(s) + 2 * L::AP_BYTES + ((32 * hf) * kD + row) * 4;
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 cv = ld_shared_f4(crow + 16 * c4);
-        float* mm = &m[4 * c4];
-        mm[0] = fmaf(g, mm[0], __uint_as_float(d[4 * c4 + 0])) + cv.x;
-        mm[1] = fmaf(g, mm[1], __uint_as_float(d[4 * c4 + 1])) + cv.y;
-        mm[2] = fmaf(g, mm[2], __uint_as_float(d[4 * c4 + 2])) + cv.z;
-        mm[3] = fmaf(g, mm[3], __uint_as_float(d[4 * c4 + 3])) + cv.w;
+      for (int jj = 0; jj < 32; ++jj) {
+        float cv;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(cv) : "r"(ccol + jj * kD * 4) : "memory");
+        m[jj] = fmaf(g, m[jj], __uint_as_float(d[jj])) + cv;
       }
       store_state(mch);
       if (own) store_state(mo_buf(jo & 1));
@@ -625,9 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int lrow = qd * 32 + lane;           // accumulator row = TMEM lane
     const float* gam = p.gamma + (size_t)bh * T;
     const float* bet = p.beta + (size_t)bh * T;
-    int own_n[NAC];                              // own frames filled per slot so far
-#pragma unroll
-    for (int i = 0; i < NAC; ++i) own_n[i] = 0;
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
       const int b = j & 1;
@@ -669,66 +660,73 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int i = 0; i < kD; ++i) v[i] = __float_as_uint(coef * __uint_as_float(v[i]));
       }
       const int s = f % NAC;
-      // The local slot is free once frame f - NAC has been consumed here. With one
-      // CTA per head every frame is ours and the release phases come in order;
-      // otherwise the loader hands the slot over in frame order.
-      bool slot_ok;
+      uint32_t sent = 1;
       if (P == 1) {
-        slot_ok = warp_wait(bar(L::B_AC_EMPTY + s), ((f / NAC) & 1) ^ 1, ctl, kStAcEmpty);
-      } else {
-        int n = 0;
+        // Every frame is ours: build it in the local slot once frame f - NAC is consumed.
+        if (!warp_wait(bar(L::B_AC_EMPTY + s), ((f / NAC) & 1) ^ 1, ctl, kStAcEmpty)) break;
+        if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
+        const uint32_t slot = ac_slot(s);
+        if (lrow < kD) {
+          // row lrow of A', bf16 hi + lo, K-major, 128-byte swizzle
 #pragma unroll
-        for (int i = 0; i < NAC; ++i)
-          if (i == s) n = own_n[i]++;
-        slot_ok = warp_wait(bar(L::B_OWN_FREE + s), n & 1, ctl, kStAcEmpty);
-      }
-      if (!slot_ok) break;
-      if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
-      const uint32_t slot = ac_slot(s);
-      if (lrow < kD) {
-        // row lrow of A', bf16 hi + lo, K-major, 128-byte swizzle
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t off = swz_off(lrow, c, 128, 3);
+            st_shared_v4(slot + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]));
+            st_shared_v4(slot + L::AP_BYTES + off,
+                         make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]));
+          }
+        } else {
+          // column (lrow - 64) of c = row (lrow - 64) of c^T
+          const uint32_t dst = slot + 2 * L::AP_BYTES + (lrow - kD) * kD * 4;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t off = swz_off(lrow, c, 128, 3);
-          st_shared_v4(slot + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]));
-          st_shared_v4(slot + L::AP_BYTES + off,
-                       make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]));
+          for (int i = 0; i < kD; i += 4)
+            st_shared_v4(dst + i * 4, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+        fence_proxy_async_cta();     // visible to the MMA
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
+        if (warp == 8 && lane == 0) {
+          sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+          if (sent) mbar_arrive(bar(L::B_AC_FULL + s));
+          GDN_TRACE_EV(8, j);
         }
       } else {
-        // column (lrow - 64) of c, fp32 row-major
-        const uint32_t dst = slot + 2 * L::AP_BYTES + (lrow - kD) * 4;
-#pragma unroll
-        for (int i = 0; i < kD; ++i)
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + i * kD * 4), "r"(v[i]) : "memory");
-      }
-      fence_proxy_async_cta();     // visible to the MMA and to the bulk-copy engine
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
-      uint32_t sent = 1;
-      if (warp == 8 && lane == 0) {
-        sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+        // Publish to every CTA of the head (this one included) through the ring.
+        // Its slot is free once each CTA has loaded frame f - kRing.
         const size_t rs = (size_t)bh * kRing + f % kRing;
-        if (sent && P > 1) {
-          // Publish to the other CTAs of the head through the ring: its slot is
-          // free once each of them has loaded frame f - kRing.
-          for (int q = 0; q < P && sent && f >= kRing; ++q)
-            if (q != (int)rank)
-              sent = wait_global_ge(p.ring_loaded + (size_t)bh * P + q,
-                                    (unsigned long long)(f - kRing + 1), ctl, kStRing);
+        uint32_t ok = 1;
+        if (lane == 0)
+          for (int q = 0; q < P && ok && f >= kRing; ++q)
+            ok = wait_global_ge(p.ring_loaded + (size_t)bh * P + q,
+                                (unsigned long long)(f - kRing + 1), ctl, kStRing) ? 1u : 0u;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
+        uint8_t* img = p.ring + rs * L::AC_BYTES;
+        if (lrow < kD) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t off = swz_off(lrow, c, 128, 3);
+            *reinterpret_cast<uint4*>(img + off) =
+                make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]);
+            *reinterpret_cast<uint4*>(img + L::AP_BYTES + off) =
+                make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]);
+          }
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(img + 2 * L::AP_BYTES + (lrow - kD) * kD * 4);
+#pragma unroll
+          for (int i = 0; i < kD; i += 4) dst[i / 4] = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
+        if (warp == 8 && lane == 0) {
+          sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
           if (sent) {
             fence_proxy_async_global();
-            bulk_store_global(p.ring + rs * L::AC_BYTES, slot, L::AC_BYTES);
-            bulk_commit();
-            bulk_wait_read0();     // the local slot may be consumed and reused from here on
+            st_release_gpu_u64(p.ring_flag + rs, (unsigned long long)(f + 1));
           }
+          GDN_TRACE_EV(8, j);
         }
-        if (sent) mbar_arrive(bar(L::B_AC_FULL + s));
-        if (sent && P > 1) {
-          bulk_wait0();
-          fence_proxy_async_global();
-          st_release_gpu_u64(p.ring_flag + rs, (unsigned long long)(f + 1));
-        }
-        GDN_TRACE_EV(8, j);
       }
       sent = __shfl_sync(0xffffffffu, sent, 0);   // warp-uniform verdict (other warps: abort flag)
       if (!sent) break;
