@@ -67,7 +67,7 @@ constexpr int kD = 64;
 constexpr int kTile = 128;                                      // rows per tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;                 // 16 KB
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
-constexpr int kRing = 8;                                        // frames per head in the ring
+constexpr int kRing = 16;                                       // frames per head in the ring
 
 // Status codes recorded in g_tc_status (bit per waiting role).
 enum : uint32_t {
@@ -106,7 +106,7 @@ struct Layout {
   static constexpr int B_Q_FULL = B_KV_EMPTY + NKV;
   static constexpr int B_Q_EMPTY = B_Q_FULL + NQ;
   static constexpr int B_AC_FULL = B_Q_EMPTY + NQ;      // [NAC] operands of the frame ready
-  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;    // [NAC] frame consumed locally
+  static constexpr int B_AC_EMPTY = B_AC_FULL + NAC;    // [NAC] frame consumed (recurrence warps)
   static constexpr int B_GB_FULL = B_AC_EMPTY + NAC;
   static constexpr int B_GB_FREE = B_GB_FULL + 2;
   static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     for (int i = 0; i < NAC; ++i) {
       mbar_init(bar(L::B_AC_FULL + i), 1);
-      mbar_init(bar(L::B_AC_EMPTY + i), 1);
+      mbar_init(bar(L::B_AC_EMPTY + i), 4);         // the 4 recurrence warps
       mbar_init(bar(L::B_LD_DONE + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -396,18 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     int t = 0;                         // next frame of the recurrence
     int gj = 0, gi = 0, kvit = 0;      // [G; b^T] stream: own frame, tile, ring counter
     int oj = 0, oi = 0, qit = 0, on = 0;
-    int rel = 0;                       // next frame whose transition slot is to be released
     uint64_t t0 = globaltimer_ns();
     while (t < T || gj < nown || oj < nown) {
       bool progressed = false;
-      // Frame t-1 is fully consumed once the recurrence warps finished it (its
-      // MMA completed and they read its c): its slot may be refilled.
-      if (rel < t && t < T && mbar_test(bar(L::B_M_READY), t & 1)) {
-        mbar_arrive(bar(L::B_AC_EMPTY + rel % NAC));
-        ++rel;
-        progressed = true;
-      }
-      if (t < T && rel == t && mbar_test(bar(L::B_M_READY), t & 1) &&
+      if (t < T && mbar_test(bar(L::B_M_READY), t & 1) &&
           mbar_test(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1)) {
         tc_fence_after();
         const uint32_t ac = ac_slot(t % NAC);
@@ -511,11 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     // order, so each wait below is for the next phase of its barrier.
     for (int t = 0; t < T; ++t) {
       const int s = t % NAC;
-      if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
       {
         const size_t rs = (size_t)bh * kRing + t % kRing;
         if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
         GDN_TRACE_EV(16, t);
+        if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
+        GDN_TRACE_EV(18, t);
         fence_proxy_async_global();
         int n = 0;
 #pragma unroll
@@ -528,8 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         mbar_arrive(bar(L::B_AC_FULL + s));
         GDN_TRACE_EV(17, t);
       }
-      // Frames up to t are loaded here: their ring slots may be reused.
-      st_release_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t + 1));
+      // Frames up to t are loaded here (their bulk loads completed above), so their
+      // ring slots may be reused; producers only need this 8 frames ahead, so it is
+      // published every other frame, without a release fence.
+      if ((t & 1) || t == T - 1)
+        st_relaxed_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t + 1));
       if (aborted(ctl)) break;
     }
   } else if (warp >= 4 && warp < 8) {
@@ -604,6 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
+        mbar_arrive(bar(L::B_AC_EMPTY + s));   // A'_t read by its MMA, c_t read here: slot free
         if (own) mbar_arrive(bar(L::B_MO_FULL + (jo & 1)));
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
