@@ -117,8 +117,7 @@ struct Layout {
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
-  static constexpr int B_LD_DONE = B_E1_STAGED + 2;     // [NAC] loader's bulk load landed
-  static constexpr int NBAR = B_LD_DONE + NAC;
+  static constexpr int NBAR = B_E1_STAGED + 2;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -312,7 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int i = 0; i < NAC; ++i) {
       mbar_init(bar(L::B_AC_FULL + i), 1);
       mbar_init(bar(L::B_AC_EMPTY + i), 4);         // the 4 recurrence warps
-      mbar_init(bar(L::B_LD_DONE + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
@@ -495,39 +493,30 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mma_commit(bar(L::B_DRAIN));
     drain_bar(bar(L::B_DRAIN), 0, ctl);
   } else if (warp == 3 && lane == 0 && P > 1) {
-    // ------------------------------------------------ loader of other CTAs' transition operands
-    int ldn[NAC];
-#pragma unroll
-    for (int i = 0; i < NAC; ++i) ldn[i] = 0;
+    // ------------------------------------------------ loader of the transition operands
     // Every frame, this CTA's own included, arrives through the ring, in frame
-    // order, so each wait below is for the next phase of its barrier.
-    for (int t = 0; t < T; ++t) {
+    // order, so each slot wait below is for the next phase of its barrier. The
+    // bulk load completes the slot's "full" barrier itself.
+    int t = 0;
+    for (; t < T; ++t) {
       const int s = t % NAC;
-      {
-        const size_t rs = (size_t)bh * kRing + t % kRing;
-        if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
-        GDN_TRACE_EV(16, t);
-        if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
-        GDN_TRACE_EV(18, t);
-        fence_proxy_async_global();
-        int n = 0;
-#pragma unroll
-        for (int i = 0; i < NAC; ++i)
-          if (i == s) n = ldn[i]++;
-        mbar_arrive_expect_tx(bar(L::B_LD_DONE + s), L::AC_BYTES);
-        bulk_load_global(ac_slot(s), p.ring + rs * L::AC_BYTES, L::AC_BYTES, bar(L::B_LD_DONE + s));
-        // Wait for the bytes even when aborting: the copy targets this CTA.
-        drain_bar(bar(L::B_LD_DONE + s), n & 1, ctl);
-        mbar_arrive(bar(L::B_AC_FULL + s));
-        GDN_TRACE_EV(17, t);
-      }
-      // Frames up to t are loaded here (their bulk loads completed above), so their
-      // ring slots may be reused; producers only need this 8 frames ahead, so it is
-      // published every other frame, without a release fence.
-      if ((t & 1) || t == T - 1)
-        st_relaxed_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t + 1));
-      if (aborted(ctl)) break;
+      const size_t rs = (size_t)bh * kRing + t % kRing;
+      if (!wait_global_ge(p.ring_flag + rs, (unsigned long long)(t + 1), ctl, kStRing)) break;
+      GDN_TRACE_EV(16, t);
+      if (!wait_bar(bar(L::B_AC_EMPTY + s), ((t / NAC) & 1) ^ 1, ctl, kStRing)) break;
+      GDN_TRACE_EV(18, t);
+      // Frame t - NAC has been consumed here, so its load (and every earlier one)
+      // completed: ring slots up to it may be reused by their producers.
+      if (t >= NAC)
+        st_relaxed_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t - NAC + 1));
+      fence_proxy_async_global();
+      mbar_arrive_expect_tx(bar(L::B_AC_FULL + s), L::AC_BYTES);
+      bulk_load_global(ac_slot(s), p.ring + rs * L::AC_BYTES, L::AC_BYTES, bar(L::B_AC_FULL + s));
+      GDN_TRACE_EV(17, t);
     }
+    // Loads still in flight target this CTA: let them land before it can leave.
+    for (int k = t - 1; k >= 0 && k >= t - NAC; --k)
+      drain_bar(bar(L::B_AC_FULL + k % NAC), (k / NAC) & 1, ctl);
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------ recurrence epilogue
     // The accumulator holds A' M for the 64 state rows: value columns 0-31 of
