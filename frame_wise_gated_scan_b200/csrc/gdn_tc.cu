@@ -79,7 +79,7 @@ enum : uint32_t {
 template <int P>
 struct Layout {
   static constexpr int NKV = 2;                      // K/V tile pairs in flight
-  static constexpr int NQ = 2;                       // Q tiles in flight
+  static constexpr int NQ = 3;                       // Q tiles in flight
   static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
@@ -394,6 +394,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     int t = 0;                         // next frame of the recurrence
     int gj = 0, gi = 0, kvit = 0;      // [G; b^T] stream: own frame, tile, ring counter
     int oj = 0, oi = 0, qit = 0, on = 0;
+    bool prefer_o = false;
+    auto o_ready = [&]() -> bool {
+      return mbar_test(bar(L::B_Q_FULL + qit % L::NQ), (qit / L::NQ) & 1) &&
+             mbar_test(bar(L::B_O_FREE + (on & 1)), ((on >> 1) & 1) ^ 1) &&
+             (oi > 0 || mbar_test(bar(L::B_MO_FULL + (oj & 1)), (oj >> 1) & 1));
+    };
     uint64_t t0 = globaltimer_ns();
     while (t < T || gj < nown || oj < nown) {
       bool progressed = false;
@@ -419,9 +425,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         mma_commit(bar(L::B_CHAIN_DONE));
         GDN_TRACE_EV(0, t);
         ++t;
-        progressed = true;
+        t0 = globaltimer_ns();
+        continue;                      // the recurrence has priority: poll it again first
       }
-      if (gj < nown) {
+      // At most one tile of the other two streams per pass, alternating.
+      prefer_o = !prefer_o;
+      if (gj < nown && !(prefer_o && oj < nown && o_ready())) {
         const int slot = kvit % L::NKV;
         const int b = gj & 1;
         if (mbar_test(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1) &&
@@ -448,13 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           progressed = true;
         }
       }
-      if (oj < nown) {
+      if (!progressed && oj < nown) {
         const int slot = qit % L::NQ;
         const int ob = on & 1;
         const int u = oj & 1;
-        if (mbar_test(bar(L::B_Q_FULL + slot), (qit / L::NQ) & 1) &&
-            mbar_test(bar(L::B_O_FREE + ob), ((on >> 1) & 1) ^ 1) &&
-            (oi > 0 || mbar_test(bar(L::B_MO_FULL + u), (oj >> 1) & 1))) {
+        if (o_ready()) {
           tc_fence_after();
           const uint32_t qt = q_slot(slot);
           const uint32_t mo = mo_buf(u);
