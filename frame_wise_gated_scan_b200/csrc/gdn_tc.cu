@@ -612,6 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int lrow = qd * 32 + lane;           // accumulator row = TMEM lane
     const float* gam = p.gamma + (size_t)bh * T;
     const float* bet = p.beta + (size_t)bh * T;
+    unsigned long long ring_seen = 0;            // lowest CTA progress last read (lane 0)
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
       const int b = j & 1;
@@ -688,10 +689,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // Its slot is free once each CTA has loaded frame f - kRing.
         const size_t rs = (size_t)bh * kRing + f % kRing;
         uint32_t ok = 1;
-        if (lane == 0)
-          for (int q = 0; q < P && ok && f >= kRing; ++q)
-            ok = wait_global_ge(p.ring_loaded + (size_t)bh * P + q,
-                                (unsigned long long)(f - kRing + 1), ctl, kStRing) ? 1u : 0u;
+        const unsigned long long need = (unsigned long long)(f - kRing + 1);
+        if (lane == 0 && f >= kRing && ring_seen < need) {
+          // Re-read the CTAs' progress only when the last reading no longer covers f.
+          unsigned long long lo = ~0ull;
+          for (int q = 0; q < P && ok; ++q) {
+            ok = wait_global_ge(p.ring_loaded + (size_t)bh * P + q, need, ctl, kStRing) ? 1u : 0u;
+            const unsigned long long v = ld_acquire_gpu_u64(p.ring_loaded + (size_t)bh * P + q);
+            lo = v < lo ? v : lo;
+          }
+          if (ok) ring_seen = lo;
+        }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
         uint8_t* img = p.ring + rs * L::AC_BYTES;
@@ -709,12 +717,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 #pragma unroll
           for (int i = 0; i < kD; i += 4) dst[i / 4] = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         }
-        __threadfence();
         __syncwarp();
+        if (lane == 0 && warp == 8) GDN_TRACE_EV(19, j);
         if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
         if (warp == 8 && lane == 0) {
           sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+          GDN_TRACE_EV(20, j);
           if (sent) {
+            // One fence after the CTA barrier: the release below then covers the
+            // ring writes of all four warps.
+            __threadfence();
             fence_proxy_async_global();
             st_release_gpu_u64(p.ring_flag + rs, (unsigned long long)(f + 1));
           }
