@@ -430,7 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       }
       // At most one tile of the other two streams per pass, alternating.
       prefer_o = !prefer_o;
-      if (gj < nown && !(prefer_o && oj < nown && o_ready())) {
+      const bool o_ok = oj < nown && o_ready();
+      if (gj < nown && !(prefer_o && o_ok)) {
         const int slot = kvit % L::NKV;
         const int b = gj & 1;
         if (mbar_test(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1) &&
@@ -457,11 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           progressed = true;
         }
       }
-      if (!progressed && oj < nown) {
+      if (!progressed && o_ok) {
         const int slot = qit % L::NQ;
         const int ob = on & 1;
         const int u = oj & 1;
-        if (o_ready()) {
+        {
           tc_fence_after();
           const uint32_t qt = q_slot(slot);
           const uint32_t mo = mo_buf(u);
