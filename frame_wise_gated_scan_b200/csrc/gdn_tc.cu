@@ -116,8 +116,9 @@ struct Layout {
   static constexpr int B_O_FULL = B_MO_EMPTY + 2;
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;
-  static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [2]
-  static constexpr int NBAR = B_E1_STAGED + 2;
+  static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [4] frame's A'/c written (4 warps)
+  static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
+  static constexpr int NBAR = B_PUB_DONE + 4;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -319,7 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_MO_EMPTY + i), 1);
       mbar_init(bar(L::B_O_FULL + i), 1);
       mbar_init(bar(L::B_O_FREE + i), 4);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar(L::B_E1_STAGED + i), 4);
+      mbar_init(bar(L::B_PUB_DONE + i), 1);
     }
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
@@ -366,6 +370,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     for (int k = it - 1; k >= 0 && k >= it - L::NKV; --k)
       drain_bar(bar(L::B_KV_FULL + k % L::NKV), (k / L::NKV) & 1, ctl);
+  } else if (warp == 0 && lane == 16 && P > 1) {
+    // ------------------------------------------------ publisher of this CTA's frames
+    // The fence and the release below wait for the producer warps' ring writes
+    // to be performed; doing them here keeps the producer warps streaming.
+    for (int j = 0; j < nown; ++j) {
+      const int f = (int)rank + j * P;
+      if (!wait_bar(bar(L::B_E1_STAGED + (j & 3)), (j >> 2) & 1, ctl, kStProd)) break;
+      GDN_TRACE_EV(20, j);
+      __threadfence();
+      fence_proxy_async_global();
+      st_release_gpu_u64(p.ring_flag + (size_t)bh * kRing + f % kRing, (unsigned long long)(f + 1));
+      mbar_arrive(bar(L::B_PUB_DONE + (j & 3)));
+      GDN_TRACE_EV(8, j);
+    }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ Q loader (own frames)
     int it = 0;
@@ -679,9 +697,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         fence_proxy_async_cta();     // visible to the MMA
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
+        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 3)));
         if (warp == 8 && lane == 0) {
-          sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
+          sent = wait_bar(bar(L::B_E1_STAGED + (j & 3)), (j >> 2) & 1, ctl, kStProd) ? 1u : 0u;
           if (sent) mbar_arrive(bar(L::B_AC_FULL + s));
           GDN_TRACE_EV(8, j);
         }
@@ -720,19 +738,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         __syncwarp();
         if (lane == 0 && warp == 8) GDN_TRACE_EV(19, j);
-        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 1)));
-        if (warp == 8 && lane == 0) {
-          sent = wait_bar(bar(L::B_E1_STAGED + (j & 1)), (j >> 1) & 1, ctl, kStProd) ? 1u : 0u;
-          GDN_TRACE_EV(20, j);
-          if (sent) {
-            // One fence after the CTA barrier: the release below then covers the
-            // ring writes of all four warps.
-            __threadfence();
-            fence_proxy_async_global();
-            st_release_gpu_u64(p.ring_flag + rs, (unsigned long long)(f + 1));
-          }
-          GDN_TRACE_EV(8, j);
-        }
+        // The publisher (warp 0, lane 16) fences and raises the ring flag; it must
+        // have published own frame j - 4 before its staging barrier is reused.
+        if (j >= 4 && !warp_wait(bar(L::B_PUB_DONE + (j & 3)), ((j >> 2) - 1) & 1, ctl, kStProd))
+          break;
+        if (lane == 0) mbar_arrive(bar(L::B_E1_STAGED + (j & 3)));
       }
       sent = __shfl_sync(0xffffffffu, sent, 0);   // warp-uniform verdict (other warps: abort flag)
       if (!sent) break;
