@@ -46,6 +46,9 @@ __device__ unsigned int g_tc_status = 0;
 // builds only: [rank][event][frame or own-frame index].
 constexpr int kTraceRanks = 4, kTraceEvents = 24, kTraceFrames = 1024;
 __device__ unsigned long long g_trace[kTraceRanks * kTraceEvents * kTraceFrames];
+// Recurrence issue time of every frame of the first kTraceHeads heads (rank 0).
+constexpr int kTraceHeads = 64;
+__device__ unsigned long long g_trace_heads[kTraceHeads * kTraceFrames];
 #define GDN_TRACE_EV(ev, idx)                                                              \
   do {                                                                                     \
     if (bh == 0 && (idx) < kTraceFrames)                                                   \
@@ -349,9 +352,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ K/V loader (own frames)
+    // Tiles of the next own frame are prefetched into L2 while this one loads,
+    // so the loads below see L2 latency rather than loaded-HBM latency.
+    for (int i = 0; i < ntile && (int)rank < T; ++i) {
+      tma_prefetch_3d(&p.tm_k, 0, i * kTile, bh * T + (int)rank);
+      tma_prefetch_3d(&p.tm_v, 0, i * kTile, bh * T + (int)rank);
+    }
     int it = 0;
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
+      if (j + 1 < nown)
+        for (int i = 0; i < ntile; ++i) {
+          tma_prefetch_3d(&p.tm_k, 0, i * kTile, bh * T + f + P);
+          tma_prefetch_3d(&p.tm_v, 0, i * kTile, bh * T + f + P);
+        }
       bool ok = true;
       for (int i = 0; i < ntile; ++i, ++it) {
         const int slot = it % L::NKV;
@@ -386,9 +400,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ Q loader (own frames)
+    for (int i = 0; i < ntile && (int)rank < T; ++i) tma_prefetch_3d(&p.tm_q, 0, i * kTile, bh * T + (int)rank);
     int it = 0;
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
+      if (j + 1 < nown)
+        for (int i = 0; i < ntile; ++i) tma_prefetch_3d(&p.tm_q, 0, i * kTile, bh * T + f + P);
       bool ok = true;
       for (int i = 0; i < ntile; ++i, ++it) {
         const int slot = it % L::NQ;
@@ -442,6 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         mma_commit(bar(L::B_CHAIN_DONE));
         GDN_TRACE_EV(0, t);
+#ifdef GDN_TRACE
+        if (rank == 0 && bh < kTraceHeads && t < kTraceFrames)
+          g_trace_heads[bh * kTraceFrames + t] = globaltimer_ns();
+#endif
         ++t;
         t0 = globaltimer_ns();
         continue;                      // the recurrence has priority: poll it again first
@@ -1005,6 +1026,10 @@ cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head) {
 extern "C" __attribute__((visibility("default"))) int gdn_trace_copy(void* dst, size_t bytes) {
   const size_t n = sizeof(g_trace) < bytes ? sizeof(g_trace) : bytes;
   return cudaMemcpyFromSymbol(dst, g_trace, n) == cudaSuccess ? (int)n : -1;
+}
+extern "C" __attribute__((visibility("default"))) int gdn_trace_heads_copy(void* dst, size_t bytes) {
+  const size_t n = sizeof(g_trace_heads) < bytes ? sizeof(g_trace_heads) : bytes;
+  return cudaMemcpyFromSymbol(dst, g_trace_heads, n) == cudaSuccess ? (int)n : -1;
 }
 #endif
 
