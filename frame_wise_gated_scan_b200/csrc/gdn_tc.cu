@@ -121,7 +121,8 @@ struct Layout {
   static constexpr int B_DRAIN = B_O_FREE + 2;
   static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [4] frame's A'/c written (4 warps)
   static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
-  static constexpr int NBAR = B_PUB_DONE + 4;
+  static constexpr int B_STAGE = B_PUB_DONE + 4;        // [2] output tile staged (4 warps)
+  static constexpr int NBAR = B_STAGE + 2;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
   static constexpr uint32_t BYTES = OFF_ABORT + 16;
@@ -143,6 +144,7 @@ struct TcParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  CUtensorMap tm_o;
   const float* gamma;
   const float* beta;
   const float* state_in;
@@ -328,6 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       mbar_init(bar(L::B_E1_STAGED + i), 4);
       mbar_init(bar(L::B_PUB_DONE + i), 1);
     }
+    mbar_init(bar(L::B_STAGE + 0), 4);
+    mbar_init(bar(L::B_STAGE + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
     mbar_init(bar(L::B_DRAIN), 1);
@@ -338,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
+    prefetch_tmap(&p.tm_o);
   }
   if (warp == 2) {
     tmem_alloc(tmem_ptr, L::TMEM_COLS);
@@ -515,7 +520,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
             mma_bf16(dO, a, bL, id_o, 1u);
           }
-          mma_commit(bar(L::B_Q_EMPTY + slot));
           mma_commit(bar(L::B_O_FULL + ob));
           if (oi == 0) GDN_TRACE_EV(15, oj);
           ++qit;
@@ -769,9 +773,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       if (!sent) break;
     }
   } else if (warp >= 12) {
-    // ------------------------------------------------ output tiles: TMEM -> bf16 -> global
+    // ------------------------------------------------ output tiles: TMEM -> bf16 -> TMA store
+    // Each tile is staged in the Q slot it was computed from (its MMA is done)
+    // and written with a bulk tensor store; the slot is handed back to the Q
+    // loader once the store has read it. Bulk stores keep the SM's generic
+    // write queue short, so the GPU-scope fences elsewhere stay cheap.
     const int qd = warp & 3;
     const int lrow = qd * 32 + lane;           // tile row = TMEM lane
+    const bool leader = (warp == 12 && lane == 0);
     int n = 0;
     bool ok = true;
     for (int j = 0; j < nown && ok; ++j) {
@@ -794,26 +803,45 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         tmem_wait_ld();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_O_FREE + ob));
         // All MMAs reading this frame's state are done: its buffer may be refilled.
-        if (i == ntile - 1 && warp == 12 && lane == 0) mbar_arrive(bar(L::B_MO_EMPTY + (j & 1)));
-        const int grow = i * kTile + lrow;
-        if (grow < p.S) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)bh * T + f) * p.S + grow) * kD);
+        if (i == ntile - 1 && leader) mbar_arrive(bar(L::B_MO_EMPTY + (j & 1)));
+        const int slot = n % L::NQ;            // the Q tile this output came from
+        const uint32_t tile = q_slot(slot);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-            w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-            w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-            w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-            dst[c] = w;
-          }
+        for (int c = 0; c < 8; ++c) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+          w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+          w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+          w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+          st_shared_v4(tile + swz_off(lrow, c, 128, 3), w);
         }
-        if (i == ntile - 1 && lane == 0 && warp == 12) GDN_TRACE_EV(10, j);
+        fence_proxy_async_cta();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(L::B_STAGE + (n & 1)));
+          // Only now free the accumulator: tile n + 2 (same staging barrier) cannot
+          // start before all four warps have staged tile n.
+          mbar_arrive(bar(L::B_O_FREE + ob));
+        }
+        uint32_t stored = 1;
+        if (leader) {
+          stored = wait_bar(bar(L::B_STAGE + (n & 1)), (n >> 1) & 1, ctl, kStOut) ? 1u : 0u;
+          if (stored) {
+            tma_store_3d(&p.tm_o, tile, 0, i * kTile, bh * T + f);
+            bulk_commit();
+            bulk_wait_read0();
+            mbar_arrive(bar(L::B_Q_EMPTY + slot));
+          }
+          if (i == ntile - 1) GDN_TRACE_EV(10, j);
+        }
+        if (!__shfl_sync(0xffffffffu, stored, 0)) {
+          ok = false;
+          break;
+        }
       }
     }
+    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
@@ -930,7 +958,7 @@ cudaError_t launch_p(const Problem& pr) {
   TcParams p;
   const long long frames = (long long)pr.B * pr.H * pr.T;
   if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames) ||
-      !make_map(&p.tm_v, pr.v, pr.S, frames))
+      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames))
     return cudaErrorInvalidValue;
   unsigned int* status = status_word();
   if (!status) return cudaErrorInvalidDevice;
