@@ -22,9 +22,11 @@
 //    MMA operand of the next frame;
 //  * each CTA sends its slice of M_t to the owner of frame t, which computes
 //    O_t = Q_t M_t (M in bf16 hi + lo, two MMAs) and stores it.
-// Warp roles (512 threads): 0 K/V loader, 1 Q loader, 2 MMA issuer (and TMEM
-// allocation), 3 forwarder (state slices to frame owners), 4-7 recurrence
-// epilogue, 8-11 A'/c epilogue, 12-15 output epilogue.
+// Warp roles (512 threads): warp 0 K/V loader (lane 0) and ring publisher
+// (lane 16); warp 1 Q loader (lane 0) and [K V]^T K MMA issuer (lane 16); warp 2
+// recurrence MMA issuer (lane 0, and TMEM allocation); warp 3 ring loader
+// (lane 0) and read-out MMA issuer (lane 16); warps 4-7 recurrence epilogue;
+// 8-11 A'/c epilogue; 12-15 output epilogue.
 //
 // Every wait is bounded (kTimeoutNs). A wait that runs out sets the device
 // status word and an abort flag in every CTA of the cluster; the other roles
@@ -118,8 +120,8 @@ struct Layout {
   static constexpr int B_MO_EMPTY = B_MO_FULL + 2;
   static constexpr int B_O_FULL = B_MO_EMPTY + 2;
   static constexpr int B_O_FREE = B_O_FULL + 2;
-  static constexpr int B_DRAIN = B_O_FREE + 2;
-  static constexpr int B_E1_STAGED = B_DRAIN + 1;       // [4] frame's A'/c written (4 warps)
+  static constexpr int B_DRAIN = B_O_FREE + 2;         // [3] one per MMA issuer
+  static constexpr int B_E1_STAGED = B_DRAIN + 3;       // [4] frame's A'/c written (4 warps)
   static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
   static constexpr int B_STAGE = B_PUB_DONE + 4;        // [2] output tile staged (4 warps)
   static constexpr int NBAR = B_STAGE + 2;
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mbar_init(bar(L::B_STAGE + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
-    mbar_init(bar(L::B_DRAIN), 1);
+    for (int i = 0; i < 3; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
   }
@@ -427,122 +429,105 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
       drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
   } else if (warp == 2 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
+    // ------------------------------------------------ recurrence MMA issuer
+    // tcgen05.commit tracks the MMAs of the issuing thread, so each of the three
+    // MMA streams has its own issuer and waits only on its own inputs.
     constexpr uint32_t id_chain = idesc_bf16(64, 32, 0, 1);    // A' K-major, M half MN-major
-    constexpr uint32_t id_gb = idesc_bf16(128, 64, 1, 1);      // [K V]^T and K, both MN-major
-    constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);       // Q K-major, M MN-major
-    int t = 0;                         // next frame of the recurrence
-    int gj = 0, gi = 0, kvit = 0;      // [G; b^T] stream: own frame, tile, ring counter
-    int oj = 0, oi = 0, qit = 0, on = 0;
-    bool prefer_o = false;
-    auto o_ready = [&]() -> bool {
-      return mbar_test(bar(L::B_Q_FULL + qit % L::NQ), (qit / L::NQ) & 1) &&
-             mbar_test(bar(L::B_O_FREE + (on & 1)), ((on >> 1) & 1) ^ 1) &&
-             (oi > 0 || mbar_test(bar(L::B_MO_FULL + (oj & 1)), (oj >> 1) & 1));
-    };
-    uint64_t t0 = globaltimer_ns();
-    while (t < T || gj < nown || oj < nown) {
-      bool progressed = false;
-      if (t < T && mbar_test(bar(L::B_M_READY), t & 1) &&
-          mbar_test(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1)) {
-        tc_fence_after();
-        const uint32_t ac = ac_slot(t % NAC);
+    for (int t = 0; t < T; ++t) {
+      if (!wait_bar(bar(L::B_M_READY), t & 1, ctl, kStMma) ||
+          !wait_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma))
+        break;
+      tc_fence_after();
+      const uint32_t ac = ac_slot(t % NAC);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
-            const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
-            const uint32_t mb = mch + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
-            const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
-            const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
-            mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
-            mma_bf16(dt, aH, bL, id_chain, 1u);
-            mma_bf16(dt, aL, bH, id_chain, 1u);
-          }
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
+          const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
+          const uint32_t mb = mch + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
+          const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
+          const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
+          mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
+          mma_bf16(dt, aH, bL, id_chain, 1u);
+          mma_bf16(dt, aL, bH, id_chain, 1u);
         }
-        mma_commit(bar(L::B_CHAIN_DONE));
-        GDN_TRACE_EV(0, t);
+      }
+      mma_commit(bar(L::B_CHAIN_DONE));
+      GDN_TRACE_EV(0, t);
 #ifdef GDN_TRACE
-        if (rank == 0 && bh < kTraceHeads && t < kTraceFrames)
-          g_trace_heads[bh * kTraceFrames + t] = globaltimer_ns();
+      if (rank == 0 && bh < kTraceHeads && t < kTraceFrames)
+        g_trace_heads[bh * kTraceFrames + t] = globaltimer_ns();
 #endif
-        ++t;
-        t0 = globaltimer_ns();
-        continue;                      // the recurrence has priority: poll it again first
-      }
-      // At most one tile of the other two streams per pass, alternating.
-      prefer_o = !prefer_o;
-      const bool o_ok = oj < nown && o_ready();
-      if (gj < nown && !(prefer_o && o_ok)) {
+    }
+    mma_commit(bar(L::B_DRAIN + 0));
+    drain_bar(bar(L::B_DRAIN + 0), 0, ctl);
+  } else if (warp == 1 && lane == 16) {
+    // ------------------------------------------------ [K V]^T K MMA issuer (own frames)
+    constexpr uint32_t id_gb = idesc_bf16(128, 64, 1, 1);      // [K V]^T and K, both MN-major
+    int kvit = 0;
+    bool ok = true;
+    for (int j = 0; j < nown && ok; ++j) {
+      const int b = j & 1;
+      if (!wait_bar(bar(L::B_GB_FREE + b), ((j >> 1) & 1) ^ 1, ctl, kStMma)) break;
+      for (int i = 0; i < ntile; ++i, ++kvit) {
         const int slot = kvit % L::NKV;
-        const int b = gj & 1;
-        if (mbar_test(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1) &&
-            (gi > 0 || mbar_test(bar(L::B_GB_FREE + b), ((gj >> 1) & 1) ^ 1))) {
-          tc_fence_after();
-          const uint32_t kv = kv_slot(slot);
-          const uint32_t dg = tmem + L::T_GB + 64 * b;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
-            const uint64_t bd = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
-            mma_bf16(dg, a, bd, id_gb, (gi > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(L::B_KV_EMPTY + slot));
-          if (gi == ntile - 1) {
-            mma_commit(bar(L::B_GB_FULL + b));
-            GDN_TRACE_EV(14, gj);
-            gi = 0;
-            ++gj;
-          } else {
-            ++gi;
-          }
-          ++kvit;
-          progressed = true;
-        }
-      }
-      if (!progressed && o_ok) {
-        const int slot = qit % L::NQ;
-        const int ob = on & 1;
-        const int u = oj & 1;
-        {
-          tc_fence_after();
-          const uint32_t qt = q_slot(slot);
-          const uint32_t mo = mo_buf(u);
-          const uint32_t dO = tmem + L::T_O + 64 * ob;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = smem_desc(qt + kk * 32, 16, 1024, 2);
-            const uint64_t bH = smem_desc(mo + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
-            const uint64_t bL =
-                smem_desc(mo + L::M_PART + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
-            mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
-            mma_bf16(dO, a, bL, id_o, 1u);
-          }
-          mma_commit(bar(L::B_O_FULL + ob));
-          if (oi == 0) GDN_TRACE_EV(15, oj);
-          ++qit;
-          ++on;
-          if (++oi == ntile) {
-            oi = 0;
-            ++oj;
-          }
-          progressed = true;
-        }
-      }
-      if (progressed) {
-        t0 = globaltimer_ns();
-      } else {
-        if (aborted(ctl)) break;
-        if (globaltimer_ns() - t0 > kTimeoutNs) {
-          raise_abort(ctl, kStMma);
+        if (!wait_bar(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1, ctl, kStMma)) {
+          ok = false;
           break;
         }
+        tc_fence_after();
+        const uint32_t kv = kv_slot(slot);
+        const uint32_t dg = tmem + L::T_GB + 64 * b;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
+          const uint64_t bd = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
+          mma_bf16(dg, a, bd, id_gb, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(L::B_KV_EMPTY + slot));
+      }
+      if (!ok) break;
+      mma_commit(bar(L::B_GB_FULL + b));
+      GDN_TRACE_EV(14, j);
+    }
+    mma_commit(bar(L::B_DRAIN + 1));
+    drain_bar(bar(L::B_DRAIN + 1), 0, ctl);
+  } else if (warp == 3 && lane == 16) {
+    // ------------------------------------------------ read-out MMA issuer (own frames)
+    constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);       // Q K-major, M MN-major
+    int qit = 0, on = 0;
+    bool ok = true;
+    for (int j = 0; j < nown && ok; ++j) {
+      const int u = j & 1;
+      if (!wait_bar(bar(L::B_MO_FULL + u), (j >> 1) & 1, ctl, kStMma)) break;
+      for (int i = 0; i < ntile; ++i, ++qit, ++on) {
+        const int slot = qit % L::NQ;
+        const int ob = on & 1;
+        if (!wait_bar(bar(L::B_Q_FULL + slot), (qit / L::NQ) & 1, ctl, kStMma) ||
+            !wait_bar(bar(L::B_O_FREE + ob), ((on >> 1) & 1) ^ 1, ctl, kStMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qt = q_slot(slot);
+        const uint32_t mo = mo_buf(u);
+        const uint32_t dO = tmem + L::T_O + 64 * ob;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = smem_desc(qt + kk * 32, 16, 1024, 2);
+          const uint64_t bH = smem_desc(mo + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
+          const uint64_t bL = smem_desc(mo + L::M_PART + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
+          mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
+          mma_bf16(dO, a, bL, id_o, 1u);
+        }
+        mma_commit(bar(L::B_O_FULL + ob));
+        if (i == 0) GDN_TRACE_EV(15, j);
       }
     }
-    mma_commit(bar(L::B_DRAIN));
-    drain_bar(bar(L::B_DRAIN), 0, ctl);
+    mma_commit(bar(L::B_DRAIN + 2));
+    drain_bar(bar(L::B_DRAIN + 2), 0, ctl);
   } else if (warp == 3 && lane == 0 && P > 1) {
     // ------------------------------------------------ loader of the transition operands
     // Every frame, this CTA's own included, arrives through the ring, in frame
