@@ -73,6 +73,7 @@ constexpr int kTile = 128;                                      // rows per tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;                 // 16 KB
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 constexpr int kRing = 16;                                       // frames per head in the ring
+constexpr int kStoreRows = 16;                                  // rows per output store box
 
 // Status codes recorded in g_tc_status (bit per waiting role).
 enum : uint32_t {
@@ -84,7 +85,7 @@ enum : uint32_t {
 template <int P>
 struct Layout {
   static constexpr int NKV = 2;                      // K/V tile pairs in flight
-  static constexpr int NQ = 3;                       // Q tiles in flight
+  static constexpr int NQ = 4;                       // Q tiles in flight (also output staging)
   static constexpr int NAC = 2;                      // transition-operand slots
   static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
@@ -102,9 +103,8 @@ struct Layout {
   static constexpr uint32_t OFF_KV = 0;
   static constexpr uint32_t OFF_Q = OFF_KV + NKV * KV_SLOT;
   static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
-  static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // recurrence operand
-  static constexpr uint32_t OFF_MO = OFF_MCH + M_BUF;               // 2 read-out operands
-  static constexpr uint32_t OFF_BAR = OFF_MO + 2 * M_BUF;
+  static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // [2] M_t, t = 0, 1 mod 2
+  static constexpr uint32_t OFF_BAR = OFF_MCH + 2 * M_BUF;
   // barrier indices (8 bytes each)
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_KV_EMPTY = B_KV_FULL + NKV;
@@ -116,9 +116,9 @@ struct Layout {
   static constexpr int B_GB_FREE = B_GB_FULL + 2;
   static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
   static constexpr int B_M_READY = B_CHAIN_DONE + 1;
-  static constexpr int B_MO_FULL = B_M_READY + 1;
-  static constexpr int B_MO_EMPTY = B_MO_FULL + 2;
-  static constexpr int B_O_FULL = B_MO_EMPTY + 2;
+  static constexpr int B_MCH_FULL = B_M_READY + 1;      // [2] M_t written (4 warps)
+  static constexpr int B_MCH_FREE = B_MCH_FULL + 2;     // [2] read-out MMAs of M_t done
+  static constexpr int B_O_FULL = B_MCH_FREE + 2;
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;         // [3] one per MMA issuer
   static constexpr int B_E1_STAGED = B_DRAIN + 3;       // [4] frame's A'/c written (4 warps)
@@ -161,6 +161,7 @@ struct TcParams {
   int T;
   int S;
   int ntile;
+  int chunk;        // output rows per CTA (multiple of 16); CTA r owns [r*chunk, (r+1)*chunk)
   float s;     // key scale 1/sqrt(D*S)
   float s2;    // its square
 };
@@ -302,8 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   auto kv_slot = [&](int i) -> uint32_t { return sb + L::OFF_KV + i * L::KV_SLOT; };
   auto q_slot = [&](int i) -> uint32_t { return sb + L::OFF_Q + i * kTileBytes; };
   auto ac_slot = [&](int i) -> uint32_t { return sb + L::OFF_AC + i * L::AC_SLOT; };
-  auto mo_buf = [&](int i) -> uint32_t { return sb + L::OFF_MO + i * L::M_BUF; };
-  const uint32_t mch = sb + L::OFF_MCH;
+  auto mch = [&](int i) -> uint32_t { return sb + L::OFF_MCH + i * L::M_BUF; };
+  // Output rows of this CTA, in every frame, and its Q tiles.
+  const int r0 = (int)rank * p.chunk;
+  const int r1 = min(p.S, r0 + p.chunk);
+  const int nq = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
   const uint32_t tmem_ptr = sb + L::OFF_TMEM_PTR;
   Ctl ctl{sb + L::OFF_ABORT, p.status, P};
 
@@ -323,8 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
       mbar_init(bar(L::B_GB_FREE + i), 4);
-      mbar_init(bar(L::B_MO_FULL + i), 4);
-      mbar_init(bar(L::B_MO_EMPTY + i), 1);
+      mbar_init(bar(L::B_MCH_FULL + i), 4);
+      mbar_init(bar(L::B_MCH_FREE + i), 1);
       mbar_init(bar(L::B_O_FULL + i), 1);
       mbar_init(bar(L::B_O_FREE + i), 4);
     }
@@ -406,25 +410,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       GDN_TRACE_EV(8, j);
     }
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ Q loader (own frames)
-    for (int i = 0; i < ntile && (int)rank < T; ++i) tma_prefetch_3d(&p.tm_q, 0, i * kTile, bh * T + (int)rank);
+    // ------------------------------------------------ Q loader (this CTA's rows, every frame)
+    for (int i = 0; i < nq; ++i) tma_prefetch_3d(&p.tm_q, 0, r0 + i * kTile, bh * T);
     int it = 0;
-    for (int j = 0; j < nown; ++j) {
-      const int f = (int)rank + j * P;
-      if (j + 1 < nown)
-        for (int i = 0; i < ntile; ++i) tma_prefetch_3d(&p.tm_q, 0, i * kTile, bh * T + f + P);
-      bool ok = true;
-      for (int i = 0; i < ntile; ++i, ++it) {
+    bool ok = true;
+    for (int t = 0; t < T && ok; ++t) {
+      if (t + 1 < T)
+        for (int i = 0; i < nq; ++i) tma_prefetch_3d(&p.tm_q, 0, r0 + i * kTile, bh * T + t + 1);
+      for (int i = 0; i < nq; ++i, ++it) {
         const int slot = it % L::NQ;
         if (!wait_bar(bar(L::B_Q_EMPTY + slot), ((it / L::NQ) & 1) ^ 1, ctl, kStQLoad)) {
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(bar(L::B_Q_FULL + slot), kTileBytes);
-        if (i == 0) GDN_TRACE_EV(13, j);
-        tma_load_3d(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, i * kTile, bh * T + f);
+        if (i == 0) GDN_TRACE_EV(13, t / P);
+        tma_load_3d(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, r0 + i * kTile, bh * T + t);
       }
-      if (!ok) break;
     }
     for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
       drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
@@ -446,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
           const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
-          const uint32_t mb = mch + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
+          const uint32_t mb = mch((t + 1) & 1) + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;   // M_{t-1}
           const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
           const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
           mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
@@ -495,14 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mma_commit(bar(L::B_DRAIN + 1));
     drain_bar(bar(L::B_DRAIN + 1), 0, ctl);
   } else if (warp == 3 && lane == 16) {
-    // ------------------------------------------------ read-out MMA issuer (own frames)
+    // ------------------------------------------------ read-out MMA issuer (this CTA's rows)
     constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);       // Q K-major, M MN-major
     int qit = 0, on = 0;
     bool ok = true;
-    for (int j = 0; j < nown && ok; ++j) {
-      const int u = j & 1;
-      if (!wait_bar(bar(L::B_MO_FULL + u), (j >> 1) & 1, ctl, kStMma)) break;
-      for (int i = 0; i < ntile; ++i, ++qit, ++on) {
+    for (int t = 0; t < T && ok; ++t) {
+      const int u = t & 1;
+      if (!wait_bar(bar(L::B_MCH_FULL + u), (t >> 1) & 1, ctl, kStMma)) break;
+      for (int i = 0; i < nq; ++i, ++qit, ++on) {
         const int slot = qit % L::NQ;
         const int ob = on & 1;
         if (!wait_bar(bar(L::B_Q_FULL + slot), (qit / L::NQ) & 1, ctl, kStMma) ||
@@ -512,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         tc_fence_after();
         const uint32_t qt = q_slot(slot);
-        const uint32_t mo = mo_buf(u);
+        const uint32_t mo = mch(u);
         const uint32_t dO = tmem + L::T_O + 64 * ob;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -523,8 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           mma_bf16(dO, a, bL, id_o, 1u);
         }
         mma_commit(bar(L::B_O_FULL + ob));
-        if (i == 0) GDN_TRACE_EV(15, j);
+        if (i == 0 && t % P == (int)rank) GDN_TRACE_EV(15, t / P);
       }
+      if (ok) mma_commit(bar(L::B_MCH_FREE + u));   // M_t no longer read here
     }
     mma_commit(bar(L::B_DRAIN + 2));
     drain_bar(bar(L::B_DRAIN + 2), 0, ctl);
@@ -575,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         st_shared_v4(buf + L::M_PART + off, l);
       }
     };
-    store_state(mch);                          // M_{-1} = M_0, read by the first MMA
+    store_state(mch(1));                       // M_{-1} = M_0, read by the first MMA
     fence_proxy_async_cta();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::B_M_READY));
@@ -587,12 +590,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
-      const bool own = (t % P) == (int)rank;
-      const int jo = t / P;
       const bool acok = warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain);
       if (acok && lane == 0 && warp == 4) GDN_TRACE_EV(21, t);
+      // M_t goes to buffer t % 2, which held M_{t-2}: its read-out MMAs must be done.
       if (!acok || !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
-          (own && !warp_wait(bar(L::B_MO_EMPTY + (jo & 1)), ((jo >> 1) & 1) ^ 1, ctl, kStMoEmpty))) {
+          !warp_wait(bar(L::B_MCH_FREE + (t & 1)), ((t >> 1) & 1) ^ 1, ctl, kStMoEmpty)) {
         ok = false;
         break;
       }
@@ -618,19 +620,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         asm volatile("ld.shared.f32 %0, [%1];" : "=f"(cv) : "r"(ccol + jj * kD * 4) : "memory");
         m[jj] = fmaf(g, m[jj], __uint_as_float(d[jj])) + cv;
       }
-      store_state(mch);
-      if (own) store_state(mo_buf(jo & 1));
+      store_state(mch(t & 1));
       tc_fence_before();
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
         mbar_arrive(bar(L::B_AC_EMPTY + s));   // A'_t read by its MMA, c_t read here: slot free
-        if (own) mbar_arrive(bar(L::B_MO_FULL + (jo & 1)));
+        mbar_arrive(bar(L::B_MCH_FULL + (t & 1)));   // M_t ready for the read-out
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
     }
-    if (ok && p.state_out) {
+    if (ok && p.state_out && rank == 0) {      // every CTA holds the same state
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj)
         p.state_out[((size_t)bh * kD + row) * kD + 32 * hf + jj] = m[jj];
@@ -760,23 +761,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   } else if (warp >= 12) {
     // ------------------------------------------------ output tiles: TMEM -> bf16 -> TMA store
     // Each tile is staged in the Q slot it was computed from (its MMA is done)
-    // and written with a bulk tensor store; the slot is handed back to the Q
-    // loader once the store has read it. Bulk stores keep the SM's generic
-    // write queue short, so the GPU-scope fences elsewhere stay cheap.
+    // and written with bulk tensor stores of 16 rows, this CTA's rows only; the
+    // slot goes back to the Q loader once the stores have read it. Bulk stores
+    // keep the SM's generic write queue short, so the GPU-scope fences elsewhere
+    // stay cheap.
     const int qd = warp & 3;
     const int lrow = qd * 32 + lane;           // tile row = TMEM lane
     const bool leader = (warp == 12 && lane == 0);
     int n = 0;
     bool ok = true;
-    for (int j = 0; j < nown && ok; ++j) {
-      const int f = (int)rank + j * P;
-      for (int i = 0; i < ntile; ++i, ++n) {
+    for (int t = 0; t < T && ok; ++t) {
+      for (int i = 0; i < nq; ++i, ++n) {
         const int ob = n & 1;
         if (!warp_wait(bar(L::B_O_FULL + ob), (n >> 1) & 1, ctl, kStOut)) {
           ok = false;
           break;
         }
-        if (i == 0 && lane == 0 && warp == 12) GDN_TRACE_EV(9, j);
+        if (i == 0 && lane == 0 && warp == 12 && t % P == (int)rank) GDN_TRACE_EV(9, t / P);
         tc_fence_after();
         uint32_t v[64];
 #pragma unroll
@@ -788,8 +789,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         tmem_wait_ld();
         tc_fence_before();
-        // All MMAs reading this frame's state are done: its buffer may be refilled.
-        if (i == ntile - 1 && leader) mbar_arrive(bar(L::B_MO_EMPTY + (j & 1)));
         const int slot = n % L::NQ;            // the Q tile this output came from
         const uint32_t tile = q_slot(slot);
 #pragma unroll
@@ -813,12 +812,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (leader) {
           stored = wait_bar(bar(L::B_STAGE + (n & 1)), (n >> 1) & 1, ctl, kStOut) ? 1u : 0u;
           if (stored) {
-            tma_store_3d(&p.tm_o, tile, 0, i * kTile, bh * T + f);
+            const int y0 = r0 + i * kTile;
+            const int y1 = min(r1, y0 + kTile);
+            for (int y = y0; y < y1; y += kStoreRows)
+              tma_store_3d(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, bh * T + t);
             bulk_commit();
             bulk_wait_read0();
             mbar_arrive(bar(L::B_Q_EMPTY + slot));
           }
-          if (i == ntile - 1) GDN_TRACE_EV(10, j);
+          if (i == nq - 1 && t % P == (int)rank) GDN_TRACE_EV(10, t / P);
         }
         if (!__shfl_sync(0xffffffffu, stored, 0)) {
           ok = false;
@@ -862,12 +864,12 @@ EncodeTiledFn encode_fn() {
 
 // [B*H*T][S][64] bf16 viewed as a 3-D tensor (64, S, B*H*T); 64 x 128 x 1 boxes with
 // the 128-byte swizzle. Rows past S inside a frame read as zero and are not stored.
-bool make_map(CUtensorMap* m, const void* base, int S, long long frames) {
+bool make_map(CUtensorMap* m, const void* base, int S, long long frames, int box_rows = kTile) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S, (cuuint64_t)frames};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S * kD * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)kTile, 1};
+  const cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -943,7 +945,7 @@ cudaError_t launch_p(const Problem& pr) {
   TcParams p;
   const long long frames = (long long)pr.B * pr.H * pr.T;
   if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames) ||
-      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames))
+      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames, kStoreRows))
     return cudaErrorInvalidValue;
   unsigned int* status = status_word();
   if (!status) return cudaErrorInvalidDevice;
@@ -956,6 +958,7 @@ cudaError_t launch_p(const Problem& pr) {
   p.T = pr.T;
   p.S = pr.S;
   p.ntile = (pr.S + kTile - 1) / kTile;
+  p.chunk = ((pr.S + P - 1) / P + 15) / 16 * 16;
   p.s = pr.key_scale;
   const double sd = 1.0 / ((double)kD * (double)pr.S);
   p.s2 = (float)sd;
