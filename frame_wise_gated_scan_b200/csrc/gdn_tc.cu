@@ -363,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ K/V loader (own frames)
+    // Inputs are read once: evict them first, keeping L2 for the ring and prefetches.
+    const uint64_t stream_pol = policy_evict_first();
     // Tiles of the next own frame are prefetched into L2 while this one loads,
     // so the loads below see L2 latency rather than loaded-HBM latency.
     for (int i = 0; i < ntile && (int)rank < T; ++i) {
@@ -387,9 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         mbar_arrive_expect_tx(bar(L::B_KV_FULL + slot), 2 * kTileBytes);
         if (i == 0) GDN_TRACE_EV(11, j);
         if (i == ntile - 1) GDN_TRACE_EV(12, j);
-        tma_load_3d(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kTile, bh * T + f);
-        tma_load_3d(kv_slot(slot) + kTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0, i * kTile,
-                    bh * T + f);
+        tma_load_3d_hint(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kTile, bh * T + f,
+                         stream_pol);
+        tma_load_3d_hint(kv_slot(slot) + kTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0, i * kTile,
+                         bh * T + f, stream_pol);
       }
       if (!ok) break;
     }
@@ -411,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ Q loader (this CTA's rows, every frame)
+    const uint64_t stream_pol = policy_evict_first();
     for (int i = 0; i < nq; ++i) tma_prefetch_3d(&p.tm_q, 0, r0 + i * kTile, bh * T);
     int it = 0;
     bool ok = true;
@@ -425,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         mbar_arrive_expect_tx(bar(L::B_Q_FULL + slot), kTileBytes);
         if (i == 0) GDN_TRACE_EV(13, t / P);
-        tma_load_3d(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, r0 + i * kTile, bh * T + t);
+        tma_load_3d_hint(q_slot(slot), &p.tm_q, bar(L::B_Q_FULL + slot), 0, r0 + i * kTile, bh * T + t,
+                         stream_pol);
       }
     }
     for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
@@ -536,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     // Every frame, this CTA's own included, arrives through the ring, in frame
     // order, so each slot wait below is for the next phase of its barrier. The
     // bulk load completes the slot's "full" barrier itself.
+    const uint64_t ring_pol = policy_evict_last();     // the ring (16 frames per head) stays in L2
     int t = 0;
     for (; t < T; ++t) {
       const int s = t % NAC;
@@ -550,7 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         st_relaxed_gpu_u64(p.ring_loaded + (size_t)bh * P + rank, (unsigned long long)(t - NAC + 1));
       fence_proxy_async_global();
       mbar_arrive_expect_tx(bar(L::B_AC_FULL + s), L::AC_BYTES);
-      bulk_load_global(ac_slot(s), p.ring + rs * L::AC_BYTES, L::AC_BYTES, bar(L::B_AC_FULL + s));
+      bulk_load_global_hint(ac_slot(s), p.ring + rs * L::AC_BYTES, L::AC_BYTES, bar(L::B_AC_FULL + s),
+                            ring_pol);
       GDN_TRACE_EV(17, t);
     }
     // Loads still in flight target this CTA: let them land before it can leave.
@@ -733,19 +740,22 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
         uint8_t* img = p.ring + rs * L::AC_BYTES;
+        const uint64_t ring_pol = policy_evict_last();
         if (lrow < kD) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint32_t off = swz_off(lrow, c, 128, 3);
-            *reinterpret_cast<uint4*>(img + off) =
-                make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]);
-            *reinterpret_cast<uint4*>(img + L::AP_BYTES + off) =
-                make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]);
+            st_global_v4_hint(img + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]),
+                              ring_pol);
+            st_global_v4_hint(img + L::AP_BYTES + off,
+                              make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]),
+                              ring_pol);
           }
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(img + 2 * L::AP_BYTES + (lrow - kD) * kD * 4);
+          uint8_t* dst = img + 2 * L::AP_BYTES + (lrow - kD) * kD * 4;
 #pragma unroll
-          for (int i = 0; i < kD; i += 4) dst[i / 4] = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int i = 0; i < kD; i += 4)
+            st_global_v4_hint(dst + i * 4, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]), ring_pol);
         }
         __syncwarp();
         if (lane == 0 && warp == 8) GDN_TRACE_EV(19, j);
@@ -768,6 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int qd = warp & 3;
     const int lrow = qd * 32 + lane;           // tile row = TMEM lane
     const bool leader = (warp == 12 && lane == 0);
+    const uint64_t out_pol = policy_evict_first();
     int n = 0;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
@@ -815,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             const int y0 = r0 + i * kTile;
             const int y1 = min(r1, y0 + kTile);
             for (int y = y0; y < y1; y += kStoreRows)
-              tma_store_3d(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, bh * T + t);
+              tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, bh * T + t, out_pol);
             bulk_commit();
             bulk_wait_read0();
             mbar_arrive(bar(L::B_Q_EMPTY + slot));
