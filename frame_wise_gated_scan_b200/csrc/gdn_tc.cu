@@ -71,6 +71,8 @@ constexpr int kThreads = 512;
 constexpr int kD = 64;
 constexpr int kTile = 128;                                      // rows per tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;                 // 16 KB
+constexpr int kKvRows = 64;                                     // rows per K/V tile
+constexpr uint32_t kKvTileBytes = kKvRows * kD * 2;             // 8 KB
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 constexpr int kRing = 16;                                       // frames per head in the ring
 constexpr int kStoreRows = 16;                                  // rows per output store box
@@ -84,13 +86,13 @@ enum : uint32_t {
 
 template <int P>
 struct Layout {
-  static constexpr int NKV = 2;                      // K/V tile pairs in flight
+  static constexpr int NKV = 5;                      // K/V tile pairs in flight
   static constexpr int NQ = 4;                       // Q tiles in flight (also output staging)
   static constexpr int NAC = 2;                      // transition-operand slots
-  static constexpr uint32_t KV_SLOT = 2 * kTileBytes;               // K tile, then V tile
-  static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' hi (lo follows)
+  static constexpr uint32_t KV_SLOT = 2 * kKvTileBytes;             // K tile, then V tile
+  static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' (bf16)
   static constexpr uint32_t C_BYTES = kD * kD * 4;                  // c^T, fp32: row j = column j of c
-  static constexpr uint32_t AC_BYTES = 2 * AP_BYTES + C_BYTES;      // one bulk copy
+  static constexpr uint32_t AC_BYTES = AP_BYTES + C_BYTES;          // one bulk copy
   static constexpr uint32_t AC_SLOT = align1k(AC_BYTES);
   // State operand: bf16 hi then lo, each two MN-major blocks of 32 value
   // columns (64-byte rows, 64-byte swizzle, 8-row groups of 512 bytes).
@@ -161,6 +163,7 @@ struct TcParams {
   int T;
   int S;
   int ntile;
+  int nkv;          // K/V tiles per frame (kKvRows rows each)
   int chunk;        // output rows per CTA (multiple of 16); CTA r owns [r*chunk, (r+1)*chunk)
   float s;     // key scale 1/sqrt(D*S)
   float s2;    // its square
@@ -297,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   const int bh = blockIdx.x / P;
   const int T = p.T;
   const int ntile = p.ntile;
+  const int nkv = p.nkv;
   const int nown = (T > (int)rank) ? (T - (int)rank + P - 1) / P : 0;   // frames this CTA owns
 
   auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * i; };
@@ -363,36 +367,36 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ K/V loader (own frames)
-    // Inputs are read once: evict them first, keeping L2 for the ring and prefetches.
-    const uint64_t stream_pol = policy_evict_first();
     // Tiles of the next own frame are prefetched into L2 while this one loads,
     // so the loads below see L2 latency rather than loaded-HBM latency.
-    for (int i = 0; i < ntile && (int)rank < T; ++i) {
-      tma_prefetch_3d(&p.tm_k, 0, i * kTile, bh * T + (int)rank);
-      tma_prefetch_3d(&p.tm_v, 0, i * kTile, bh * T + (int)rank);
+    // Inputs are read once: evict them first, keeping L2 for the ring and prefetches.
+    const uint64_t stream_pol = policy_evict_first();
+    for (int i = 0; i < nkv && (int)rank < T; ++i) {
+      tma_prefetch_3d(&p.tm_k, 0, i * kKvRows, bh * T + (int)rank);
+      tma_prefetch_3d(&p.tm_v, 0, i * kKvRows, bh * T + (int)rank);
     }
     int it = 0;
     for (int j = 0; j < nown; ++j) {
       const int f = (int)rank + j * P;
       if (j + 1 < nown)
-        for (int i = 0; i < ntile; ++i) {
-          tma_prefetch_3d(&p.tm_k, 0, i * kTile, bh * T + f + P);
-          tma_prefetch_3d(&p.tm_v, 0, i * kTile, bh * T + f + P);
+        for (int i = 0; i < nkv; ++i) {
+          tma_prefetch_3d(&p.tm_k, 0, i * kKvRows, bh * T + f + P);
+          tma_prefetch_3d(&p.tm_v, 0, i * kKvRows, bh * T + f + P);
         }
       bool ok = true;
-      for (int i = 0; i < ntile; ++i, ++it) {
+      for (int i = 0; i < nkv; ++i, ++it) {
         const int slot = it % L::NKV;
         if (!wait_bar(bar(L::B_KV_EMPTY + slot), ((it / L::NKV) & 1) ^ 1, ctl, kStKvLoad)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(L::B_KV_FULL + slot), 2 * kTileBytes);
+        mbar_arrive_expect_tx(bar(L::B_KV_FULL + slot), 2 * kKvTileBytes);
         if (i == 0) GDN_TRACE_EV(11, j);
-        if (i == ntile - 1) GDN_TRACE_EV(12, j);
-        tma_load_3d_hint(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kTile, bh * T + f,
+        if (i == nkv - 1) GDN_TRACE_EV(12, j);
+        tma_load_3d_hint(kv_slot(slot), &p.tm_k, bar(L::B_KV_FULL + slot), 0, i * kKvRows, bh * T + f,
                          stream_pol);
-        tma_load_3d_hint(kv_slot(slot) + kTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0, i * kTile,
-                         bh * T + f, stream_pol);
+        tma_load_3d_hint(kv_slot(slot) + kKvTileBytes, &p.tm_v, bar(L::B_KV_FULL + slot), 0,
+                         i * kKvRows, bh * T + f, stream_pol);
       }
       if (!ok) break;
     }
@@ -451,14 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
+          // A' M_{t-1} = A' M_hi + A' M_lo: A' is small next to the exact fp32
+          // gamma M term, so one bf16 copy of it suffices.
           const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
-          const uint64_t aL = smem_desc(ac + L::AP_BYTES + kk * 32, 16, 1024, 2);
           const uint32_t mb = mch((t + 1) & 1) + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;   // M_{t-1}
           const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
           const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
           mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
           mma_bf16(dt, aH, bL, id_chain, 1u);
-          mma_bf16(dt, aL, bH, id_chain, 1u);
         }
       }
       mma_commit(bar(L::B_CHAIN_DONE));
@@ -478,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int j = 0; j < nown && ok; ++j) {
       const int b = j & 1;
       if (!wait_bar(bar(L::B_GB_FREE + b), ((j >> 1) & 1) ^ 1, ctl, kStMma)) break;
-      for (int i = 0; i < ntile; ++i, ++kvit) {
+      for (int i = 0; i < nkv; ++i, ++kvit) {
         const int slot = kvit % L::NKV;
         if (!wait_bar(bar(L::B_KV_FULL + slot), (kvit / L::NKV) & 1, ctl, kStMma)) {
           ok = false;
@@ -488,9 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         const uint32_t kv = kv_slot(slot);
         const uint32_t dg = tmem + L::T_GB + 64 * b;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
-          const uint64_t bd = smem_desc(kv + kk * 2048, kTileBytes, 1024, 2);
+        for (int kk = 0; kk < kKvRows / 16; ++kk) {
+          const uint64_t a = smem_desc(kv + kk * 2048, kKvTileBytes, 1024, 2);
+          const uint64_t bd = smem_desc(kv + kk * 2048, kKvTileBytes, 1024, 2);
           mma_bf16(dg, a, bd, id_gb, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(L::B_KV_EMPTY + slot));
@@ -620,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
       }
       // c[row][32hf + jj] = c^T[32hf + jj][row]
-      const uint32_t ccol = ac_slot(s) + 2 * L::AP_BYTES + ((32 * hf) * kD + row) * 4;
+      const uint32_t ccol = ac_slot(s) + L::AP_BYTES + ((32 * hf) * kD + row) * 4;
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
         float cv;
@@ -671,8 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_GB_FREE + b));
       // Convert first, then wait for the slot: after the wait only stores remain.
-      // A' rows are packed in place: chunk c (8 values) becomes its 4 hi words
-      // in v[8c..8c+3] and its 4 lo words in v[8c+4..8c+7].
+      // A' rows are packed in place: chunk c (8 values) becomes 4 bf16x2 words in
+      // v[8c..8c+3].
       if (lrow < kD) {
         const float coef = -g * be * p.s2;       // A' = -gamma beta s^2 G
 #pragma unroll
@@ -680,10 +684,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = coef * __uint_as_float(v[8 * c + e]);
-          uint4 h, l;
-          split8(x, h, l);
-          v[8 * c + 0] = h.x; v[8 * c + 1] = h.y; v[8 * c + 2] = h.z; v[8 * c + 3] = h.w;
-          v[8 * c + 4] = l.x; v[8 * c + 5] = l.y; v[8 * c + 6] = l.z; v[8 * c + 7] = l.w;
+          v[8 * c + 0] = pack_bf16x2(x[0], x[1]);
+          v[8 * c + 1] = pack_bf16x2(x[2], x[3]);
+          v[8 * c + 2] = pack_bf16x2(x[4], x[5]);
+          v[8 * c + 3] = pack_bf16x2(x[6], x[7]);
         }
       } else {
         const float coef = be * p.s;             // c = beta s K^T V
@@ -703,12 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           for (int c = 0; c < 8; ++c) {
             const uint32_t off = swz_off(lrow, c, 128, 3);
             st_shared_v4(slot + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]));
-            st_shared_v4(slot + L::AP_BYTES + off,
-                         make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]));
           }
         } else {
           // column (lrow - 64) of c = row (lrow - 64) of c^T
-          const uint32_t dst = slot + 2 * L::AP_BYTES + (lrow - kD) * kD * 4;
+          const uint32_t dst = slot + L::AP_BYTES + (lrow - kD) * kD * 4;
 #pragma unroll
           for (int i = 0; i < kD; i += 4)
             st_shared_v4(dst + i * 4, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]));
@@ -747,12 +749,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             const uint32_t off = swz_off(lrow, c, 128, 3);
             st_global_v4_hint(img + off, make_uint4(v[8 * c], v[8 * c + 1], v[8 * c + 2], v[8 * c + 3]),
                               ring_pol);
-            st_global_v4_hint(img + L::AP_BYTES + off,
-                              make_uint4(v[8 * c + 4], v[8 * c + 5], v[8 * c + 6], v[8 * c + 7]),
-                              ring_pol);
           }
         } else {
-          uint8_t* dst = img + 2 * L::AP_BYTES + (lrow - kD) * kD * 4;
+          uint8_t* dst = img + L::AP_BYTES + (lrow - kD) * kD * 4;
 #pragma unroll
           for (int i = 0; i < kD; i += 4)
             st_global_v4_hint(dst + i * 4, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]), ring_pol);
@@ -955,8 +954,8 @@ cudaError_t launch_p(const Problem& pr) {
   if (e != cudaSuccess) return e;
   TcParams p;
   const long long frames = (long long)pr.B * pr.H * pr.T;
-  if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames) ||
-      !make_map(&p.tm_v, pr.v, pr.S, frames) || !make_map(&p.tm_o, pr.out, pr.S, frames, kStoreRows))
+  if (!make_map(&p.tm_q, pr.q, pr.S, frames) || !make_map(&p.tm_k, pr.k, pr.S, frames, kKvRows) ||
+      !make_map(&p.tm_v, pr.v, pr.S, frames, kKvRows) || !make_map(&p.tm_o, pr.out, pr.S, frames, kStoreRows))
     return cudaErrorInvalidValue;
   unsigned int* status = status_word();
   if (!status) return cudaErrorInvalidDevice;
@@ -969,6 +968,7 @@ cudaError_t launch_p(const Problem& pr) {
   p.T = pr.T;
   p.S = pr.S;
   p.ntile = (pr.S + kTile - 1) / kTile;
+  p.nkv = (pr.S + kKvRows - 1) / kKvRows;
   p.chunk = ((pr.S + P - 1) / P + 15) / 16 * 16;
   p.s = pr.key_scale;
   const double sd = 1.0 / ((double)kD * (double)pr.S);
