@@ -498,11 +498,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
           mma_bf16(dg, a, bd, id_gb, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(L::B_KV_EMPTY + slot));
-        // One tile in flight: the recurrence's MMAs never queue behind more.
-        if (!wait_bar(bar(L::B_KV_EMPTY + slot), (kvit / L::NKV) & 1, ctl, kStMma)) {
-          ok = false;
-          break;
-        }
       }
       if (!ok) break;
       mma_commit(bar(L::B_GB_FULL + b));
@@ -540,11 +535,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         mma_commit(bar(L::B_O_FULL + ob));
         if (i == 0 && t % P == (int)rank) GDN_TRACE_EV(15, t / P);
-        // One tile in flight: the recurrence's MMAs never queue behind more.
-        if (!wait_bar(bar(L::B_O_FULL + ob), (on >> 1) & 1, ctl, kStMma)) {
-          ok = false;
-          break;
-        }
       }
       if (ok) mma_commit(bar(L::B_MCH_FREE + u));   // M_t no longer read here
     }
