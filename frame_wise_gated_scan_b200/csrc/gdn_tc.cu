@@ -236,6 +236,26 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ct
   }
 }
 
+// Bounded poll with a short sleep between tests, for the recurrence's
+// latency-critical handoffs: it reacts within tens of nanoseconds without
+// taking issue slots from the other warps of its sub-partition.
+__device__ __forceinline__ bool poll_bar(uint32_t bar, uint32_t parity, const Ctl& c,
+                                         uint32_t code) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i) {
+      __nanosleep(20);
+      if (mbar_test(bar, parity)) return true;
+    }
+    if (aborted(c)) return false;
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      raise_abort(c, code);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, and on
 // success every lane observes the completed phase itself (acquire).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl& c,
@@ -445,8 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     // MMA streams has its own issuer and waits only on its own inputs.
     constexpr uint32_t id_chain = idesc_bf16(64, 32, 0, 1);    // A' K-major, M half MN-major
     for (int t = 0; t < T; ++t) {
-      if (!wait_bar(bar(L::B_M_READY), t & 1, ctl, kStMma) ||
-          !wait_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma))
+      if (!poll_bar(bar(L::B_M_READY), t & 1, ctl, kStMma) ||
+          !poll_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma))
         break;
       tc_fence_after();
       const uint32_t ac = ac_slot(t % NAC);
@@ -604,7 +624,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const bool acok = warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain);
       if (acok && lane == 0 && warp == 4) GDN_TRACE_EV(21, t);
       // M_t goes to buffer t % 2, which held M_{t-2}: its read-out MMAs must be done.
-      if (!acok || !warp_wait(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ||
+      uint32_t cd = 0;
+      if (acok && lane == 0) cd = poll_bar(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ? 1u : 0u;
+      cd = __shfl_sync(0xffffffffu, cd, 0);
+      if (cd) mbar_test(bar(L::B_CHAIN_DONE), t & 1);    // acquire for every lane
+      if (!acok || !cd ||
           !warp_wait(bar(L::B_MCH_FREE + (t & 1)), ((t >> 1) & 1) ^ 1, ctl, kStMoEmpty)) {
         ok = false;
         break;
