@@ -23,7 +23,13 @@
  *
  * Pointers: every array pointer is a DEVICE pointer of the current CUDA
  * device. The caller owns every buffer; the library keeps no pointer after a
- * call returns and allocates no device memory. q, k, v, out, state_in and
+ * call returns. Device memory: a bf16 scan that runs the tensor-core kernel
+ * with more than one CTA per head (see gdn_plan) takes stream-ordered scratch
+ * for the transition operands the CTAs of a head share (16 frames x 24 KiB
+ * per head, plus 8 bytes x (16 + CTAs per head) of flags), with
+ * cudaMallocAsync on `stream`, and releases it with cudaFreeAsync on the same
+ * stream right after the launch; every other call allocates no device
+ * memory. q, k, v, out, state_in and
  * state_out must be 16-byte aligned; gamma and beta 4-byte aligned.
  * state_in == NULL means M_0 = 0. state_out == NULL means the final state is
  * not written. state_in may equal state_out (the update is then in place);
