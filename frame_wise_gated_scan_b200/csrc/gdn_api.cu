@@ -51,9 +51,10 @@ int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
 
 int run(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
         const float* state_in, float* state_out, void* out, int B, int H, int T, int S, int D,
-        void* stream, int elt_bytes) {
+        void* stream, int elt_bytes, bool noalloc = false) {
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
+  if (noalloc && (long long)B * H > GDN_NOALLOC_MAX_HEADS) return GDN_ERR_SCRATCH;
   if (!q || !k || !v || !gamma || !beta || !out) return GDN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(gamma, 4) ||
@@ -90,7 +91,10 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   } else {
     int ctas = 1;
     const int kern = choose_kernel(B, H, T, S, D, &ctas);
-    err = (kern == GDN_KERNEL_TC) ? gdn::launch_tc_bf16(p, ctas) : gdn::launch_simt_bf16(p);
+    if (kern != GDN_KERNEL_TC)
+      err = gdn::launch_simt_bf16(p);   // allocates nothing either way
+    else
+      err = noalloc ? gdn::launch_tc_bf16_noalloc(p, ctas) : gdn::launch_tc_bf16(p, ctas);
   }
   return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -103,6 +107,12 @@ int gdn_frame_scan(const void* q, const void* k, const void* v, const float* gam
                    const float* beta, const float* state_in, float* state_out, void* out, int B,
                    int H, int T, int S, int D, void* stream) {
   return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 2);
+}
+
+int gdn_frame_scan_noalloc(const void* q, const void* k, const void* v, const float* gamma,
+                           const float* beta, const float* state_in, float* state_out, void* out,
+                           int B, int H, int T, int S, int D, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 2, true);
 }
 
 int gdn_frame_step(const void* q, const void* k, const void* v, const float* gamma,
@@ -148,6 +158,8 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "a CUDA call failed";
     case GDN_ERR_TIMEOUT: return "a device-side wait ran out; outputs of that call are incomplete";
     case GDN_ERR_ALIAS: return "out overlaps an input or a state buffer";
+    case GDN_ERR_SCRATCH:
+      return "B * H exceeds GDN_NOALLOC_MAX_HEADS (32), the fixed scratch of gdn_frame_scan_noalloc";
     default: return "unknown gdn_status";
   }
 }

@@ -30,6 +30,10 @@ cudaError_t launch_simt_bf16(const Problem& p);
 // or 0 if it does not take them.
 int tc_ctas_per_head(int B, int H, int T, int S, int D);
 cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head);
+// The same kernel with its scratch taken from a fixed device array instead of
+// stream-ordered allocations (gdn_frame_scan_noalloc). Needs B * H <=
+// GDN_NOALLOC_MAX_HEADS; calls that overlap on the GPU race on the array.
+cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head);
 // Reads and clears the device status word of the tensor-core kernel.
 cudaError_t tc_read_status(unsigned int* status);
 

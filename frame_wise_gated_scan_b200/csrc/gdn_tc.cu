@@ -36,6 +36,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <atomic>
+
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "sm100_ptx.h"
 
@@ -143,6 +146,17 @@ struct Layout {
 static_assert(Layout<4>::SMEM_ALLOC <= 232448, "shared memory budget (P=4)");
 static_assert(Layout<2>::SMEM_ALLOC <= 232448, "shared memory budget (P=2)");
 static_assert(Layout<1>::SMEM_ALLOC <= 232448, "shared memory budget (P=1)");
+
+// Scratch of gdn_frame_scan_noalloc, for callers that cannot allocate: the
+// ring and its flags (TcParams below) for up to GDN_NOALLOC_MAX_HEADS heads at
+// the largest cluster size, 12 MiB + 5 KiB. The ring starts at the base, the
+// flags at kNoAllocRingBytes.
+constexpr size_t kNoAllocRingBytes = (size_t)GDN_NOALLOC_MAX_HEADS * kRing * Layout<4>::AC_BYTES;
+constexpr size_t kNoAllocFlagBytes =
+    (size_t)GDN_NOALLOC_MAX_HEADS * (kRing + 4) * sizeof(unsigned long long);
+static_assert(Layout<2>::AC_BYTES == Layout<4>::AC_BYTES, "one ring image size for every P");
+static_assert(kNoAllocRingBytes % 256 == 0, "flags stay aligned");
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocRingBytes + kNoAllocFlagBytes];
 
 struct TcParams {
   CUtensorMap tm_q;
@@ -972,8 +986,31 @@ unsigned int* status_word() {
   return cache[dev];
 }
 
+// Address of g_noalloc_scratch on the current device. cudaGetSymbolAddress
+// (which allocates nothing) runs once per device, with that device current;
+// the address is kept for later calls.
+cudaError_t noalloc_scratch(uint8_t** out) {
+  static std::atomic<uint8_t*> cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  uint8_t* a = cache[dev].load(std::memory_order_acquire);
+  if (!a) {
+    void* sym = nullptr;
+    e = cudaGetSymbolAddress(&sym, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    a = static_cast<uint8_t*>(sym);
+    cache[dev].store(a, std::memory_order_release);
+  }
+  *out = a;
+  return cudaSuccess;
+}
+
+// fixed_scratch: null for gdn_frame_scan (stream-ordered scratch when P > 1),
+// g_noalloc_scratch's address for gdn_frame_scan_noalloc.
 template <int P>
-cudaError_t launch_p(const Problem& pr) {
+cudaError_t launch_p(const Problem& pr, uint8_t* fixed_scratch) {
   cudaError_t e = prepare<P>();
   if (e != cudaSuccess) return e;
   TcParams p;
@@ -1007,7 +1044,15 @@ cudaError_t launch_p(const Problem& pr) {
   p.ring = nullptr;
   p.ring_flag = nullptr;
   p.ring_loaded = nullptr;
-  if (P > 1) {
+  if (P > 1 && fixed_scratch) {
+    // The fixed array: nothing to allocate; its flags must start at zero.
+    if (heads > (size_t)GDN_NOALLOC_MAX_HEADS) return cudaErrorInvalidValue;
+    p.ring = fixed_scratch;
+    p.ring_flag = reinterpret_cast<unsigned long long*>(fixed_scratch + kNoAllocRingBytes);
+    p.ring_loaded = p.ring_flag + heads * kRing;
+    e = cudaMemsetAsync(p.ring_flag, 0, ctrl_bytes, pr.stream);
+    if (e != cudaSuccess) return e;
+  } else if (P > 1) {
     e = cudaMallocAsync(&scratch, ring_bytes + ctrl_bytes, pr.stream);
     if (e != cudaSuccess) return e;
     p.ring = static_cast<uint8_t*>(scratch);
@@ -1066,9 +1111,22 @@ int tc_ctas_per_head(int B, int H, int T, int S, int D) {
 
 cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head) {
   switch (ctas_per_head) {
-    case 1: return launch_p<1>(p);
-    case 2: return launch_p<2>(p);
-    case 4: return launch_p<4>(p);
+    case 1: return launch_p<1>(p, nullptr);
+    case 2: return launch_p<2>(p, nullptr);
+    case 4: return launch_p<4>(p, nullptr);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head) {
+  if ((long long)p.B * p.H > GDN_NOALLOC_MAX_HEADS) return cudaErrorInvalidValue;
+  if (ctas_per_head == 1) return launch_p<1>(p, nullptr);   // no ring, no scratch
+  uint8_t* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  switch (ctas_per_head) {
+    case 2: return launch_p<2>(p, scratch);
+    case 4: return launch_p<4>(p, scratch);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         scan_args = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
         step_args = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, vp]
         for name, args in (("gdn_frame_scan", scan_args), ("gdn_frame_scan_f32", scan_args),
+                           ("gdn_frame_scan_noalloc", scan_args),
                            ("gdn_frame_step", step_args), ("gdn_frame_step_f32", step_args)):
             fn = getattr(L, name)
             fn.argtypes = args
@@ -106,7 +107,8 @@ def _check(t, name, dtype, shape, device):
         raise ValueError(f"{name}: must be contiguous")
 
 
-def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state):
+def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state,
+          noalloc=False):
     if q.dim() != (4 if step else 5):
         raise ValueError("q must be [B,H,S,D] for a step, [B,H,T,S,D] for a scan")
     device = q.device
@@ -142,7 +144,9 @@ def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state
     if not step:
         args.append(T)
     args += [S, D, _stream_handle(device)]
-    if step:
+    if noalloc:
+        fn = L.gdn_frame_scan_noalloc
+    elif step:
         fn = L.gdn_frame_step if dt == torch.bfloat16 else L.gdn_frame_step_f32
     else:
         fn = L.gdn_frame_scan if dt == torch.bfloat16 else L.gdn_frame_scan_f32
@@ -160,6 +164,19 @@ def frame_scan(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
     Returns (out, state_out); state_out is None if want_state is False and
     none was given."""
     return _call(False, q, k, v, gamma, beta, state_in, out, state_out, want_state)
+
+
+def frame_scan_noalloc(q, k, v, gamma, beta, state_in=None, *, out, state_out=None):
+    """frame_scan through gdn_frame_scan_noalloc, for callers that must not
+    allocate device memory: bf16 only, B*H <= 32, and out (plus state_out, if
+    the final state is wanted) supplied by the caller, so nothing is allocated
+    here either. Calls on one device must not overlap on the GPU: they share
+    the library's fixed scratch."""
+    if q.dtype != torch.bfloat16:
+        raise TypeError("frame_scan_noalloc takes bfloat16 q, k, v")
+    if q.dim() != 5:
+        raise ValueError("q must be [B,H,T,S,D]")
+    return _call(False, q, k, v, gamma, beta, state_in, out, state_out, False, noalloc=True)
 
 
 def frame_step(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,

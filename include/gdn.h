@@ -69,7 +69,8 @@ typedef enum gdn_status {
   GDN_ERR_ALIGN = -4,           /* a pointer breaks the alignment rules above */
   GDN_ERR_CUDA = -5,            /* a CUDA runtime or driver call failed */
   GDN_ERR_TIMEOUT = -6,         /* a device-side wait ran out (from gdn_device_status) */
-  GDN_ERR_ALIAS = -7            /* out overlaps an input or a state buffer */
+  GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
+  GDN_ERR_SCRATCH = -8          /* B * H > GDN_NOALLOC_MAX_HEADS (gdn_frame_scan_noalloc) */
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
@@ -88,6 +89,45 @@ GDN_API int gdn_frame_step(const void* q, const void* k, const void* v,
                    const float* gamma, const float* beta,
                    const float* state_in, float* state_out, void* out,
                    int B, int H, int S, int D, void* stream);
+
+/* gdn_frame_scan for callers that must not allocate device memory. The
+ * method has no counterpart to this entry point: it exists for the library's
+ * users, not for the operation.
+ *
+ * Who needs it: a caller that has reserved nearly all of the GPU's memory for
+ * its own pool up front (an inference engine, say) cannot let a library take
+ * more during a call, since the allocation would fail or push out its cache;
+ * a process with a hard device-memory cap is in the same place; and a caller
+ * in a tight loop may not accept the cost of an allocation at all (cudaMalloc
+ * and cudaFree can synchronize the device, and a stream-ordered pool may have
+ * to grow). gdn_frame_scan takes stream-ordered scratch when it runs with
+ * more than one CTA per head; this entry point takes that scratch from one
+ * fixed array in the library's device code instead, and calls no cudaMalloc,
+ * cudaMallocAsync, cudaFree or cudaFreeAsync.
+ *
+ * Limit: B * H <= GDN_NOALLOC_MAX_HEADS (32); larger sizes return
+ * GDN_ERR_SCRATCH and enqueue nothing. The array holds 16 frames x 24 KiB of
+ * transition operands plus 160 bytes of flags per head: 12 MiB + 5 KiB,
+ * reserved on each device when the library's device code is loaded there,
+ * whether or not this entry point is called. The first call on a device looks
+ * the array's address up (cudaGetSymbolAddress, with that device current) and
+ * keeps it for later calls; every call then clears the array's flags with
+ * cudaMemsetAsync on `stream` before its kernel.
+ *
+ * Concurrency: every call on a device uses the same array. Two calls whose
+ * work overlaps on the GPU (different streams with no ordering between them,
+ * or calls from several host threads) race on it: their results are wrong or
+ * a bounded device wait runs out (gdn_device_status then reports
+ * GDN_ERR_TIMEOUT). Order such calls, on one stream or with events.
+ * gdn_frame_scan and the other entry points do not touch the array.
+ *
+ * Arguments, layouts, results and errors are those of gdn_frame_scan; for
+ * the same inputs and kernel choice (gdn_plan) the results are identical. */
+#define GDN_NOALLOC_MAX_HEADS 32
+GDN_API int gdn_frame_scan_noalloc(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int T, int S, int D, void* stream);
 
 /* float32 variants: q, k, v, out are float; every operation runs in fp32 on
  * CUDA cores (FFMA), in the definition's order (W, then R, then K^T R). */

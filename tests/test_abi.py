@@ -19,7 +19,8 @@ def L():
 def test_every_declared_symbol_is_exported(L):
     names = gdn.header_symbols()
     assert set(names) >= {"gdn_frame_scan", "gdn_frame_step", "gdn_frame_scan_f32",
-                          "gdn_frame_step_f32", "gdn_plan", "gdn_device_status",
+                          "gdn_frame_step_f32", "gdn_frame_scan_noalloc", "gdn_plan",
+                          "gdn_device_status",
                           "gdn_status_string", "gdn_version"}
     out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -33,7 +34,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strings(L):
     assert gdn.version() == 10000
-    for st in range(-7, 1):
+    for st in range(-8, 1):
         s = gdn.status_string(st)
         assert s and s != "unknown gdn_status"
     assert gdn.status_string(-99) == "unknown gdn_status"
