@@ -54,12 +54,23 @@ __device__ unsigned long long g_trace[kTraceRanks * kTraceEvents * kTraceFrames]
 // Recurrence issue time of every frame of the first kTraceHeads heads (rank 0).
 constexpr int kTraceHeads = 64;
 __device__ unsigned long long g_trace_heads[kTraceHeads * kTraceFrames];
+// Per CTA (first kTraceCtas): SM id, and the K/V loader's clock when it starts
+// its third own frame and its last one.
+constexpr int kTraceCtas = 1024;
+__device__ unsigned long long g_trace_cta[kTraceCtas * 4];
+#define GDN_TRACE_CTA(slot, value)                                     \
+  do {                                                                 \
+    if (blockIdx.x < kTraceCtas) g_trace_cta[blockIdx.x * 4 + (slot)] = (value); \
+  } while (0)
 #define GDN_TRACE_EV(ev, idx)                                                              \
   do {                                                                                     \
     if (bh == 0 && (idx) < kTraceFrames)                                                   \
       g_trace[((int)rank * kTraceEvents + (ev)) * kTraceFrames + (idx)] = globaltimer_ns(); \
   } while (0)
 #else
+#define GDN_TRACE_CTA(slot, value) \
+  do {                             \
+  } while (0)
 #define GDN_TRACE_EV(ev, idx) \
   do {                        \
   } while (0)
@@ -92,24 +103,25 @@ struct Layout {
   static constexpr int NKV = 5;                      // K/V tile pairs in flight
   static constexpr int NQ = 4;                       // Q tiles in flight (also output staging)
   static constexpr int NAC = 2;                      // transition-operand slots
+  static constexpr int NM = 4;                       // state operand buffers: M_t in t % NM
+  static constexpr int NCLAIM = 16;                  // claimed frames (jobs) in flight
   static constexpr uint32_t KV_SLOT = 2 * kKvTileBytes;             // K tile, then V tile
   static constexpr uint32_t AP_BYTES = kD * kD * 2;                 // A' (bf16)
   static constexpr uint32_t C_BYTES = kD * kD * 4;                  // c^T, fp32: row j = column j of c
   static constexpr uint32_t AC_BYTES = AP_BYTES + C_BYTES;          // one bulk copy
   static constexpr uint32_t AC_SLOT = align1k(AC_BYTES);
-  // State operand: bf16 hi then lo, each two MN-major blocks of 32 value
-  // columns (64-byte rows, 64-byte swizzle, 8-row groups of 512 bytes).
+  // State operand: M in bf16, two MN-major blocks of 32 value columns
+  // (64-byte rows, 64-byte swizzle, 8-row groups of 512 bytes).
   static constexpr uint32_t MB_RW = 64;
   static constexpr uint32_t MB_SBO = 8 * MB_RW;
   static constexpr uint32_t MB_BLOCK = kD * MB_RW;                  // 4 KB
-  static constexpr uint32_t M_PART = 2 * MB_BLOCK;                  // 8 KB
-  static constexpr uint32_t M_BUF = 2 * M_PART;                     // 16 KB
+  static constexpr uint32_t M_BUF = 2 * MB_BLOCK;                   // 8 KB
 
   static constexpr uint32_t OFF_KV = 0;
   static constexpr uint32_t OFF_Q = OFF_KV + NKV * KV_SLOT;
   static constexpr uint32_t OFF_AC = OFF_Q + NQ * kTileBytes;
-  static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // [2] M_t, t = 0, 1 mod 2
-  static constexpr uint32_t OFF_BAR = OFF_MCH + 2 * M_BUF;
+  static constexpr uint32_t OFF_MCH = OFF_AC + NAC * AC_SLOT;      // [NM] M_t in buffer t % NM
+  static constexpr uint32_t OFF_BAR = OFF_MCH + NM * M_BUF;
   // barrier indices (8 bytes each)
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_KV_EMPTY = B_KV_FULL + NKV;
@@ -121,18 +133,21 @@ struct Layout {
   static constexpr int B_GB_FREE = B_GB_FULL + 2;
   static constexpr int B_CHAIN_DONE = B_GB_FREE + 2;
   static constexpr int B_M_READY = B_CHAIN_DONE + 1;
-  static constexpr int B_MCH_FULL = B_M_READY + 1;      // [2] M_t written (4 warps)
-  static constexpr int B_MCH_FREE = B_MCH_FULL + 2;     // [2] read-out MMAs of M_t done
-  static constexpr int B_O_FULL = B_MCH_FREE + 2;
+  static constexpr int B_MCH_FULL = B_M_READY + 1;      // [NM] M_t written (4 warps)
+  static constexpr int B_MCH_FREE = B_MCH_FULL + NM;    // [NM] read-out MMAs of M_t done
+  static constexpr int B_O_FULL = B_MCH_FREE + NM;
   static constexpr int B_O_FREE = B_O_FULL + 2;
   static constexpr int B_DRAIN = B_O_FREE + 2;         // [3] one per MMA issuer
   static constexpr int B_E1_STAGED = B_DRAIN + 3;       // [4] frame's A'/c written (4 warps)
   static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
   static constexpr int B_STAGE = B_PUB_DONE + 4;        // [2] output tile staged (4 warps)
-  static constexpr int NBAR = B_STAGE + 2;
+  static constexpr int B_CLAIM = B_STAGE + 2;           // [NCLAIM] frame of job j known
+  static constexpr int NBAR = B_CLAIM + NCLAIM;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
-  static constexpr uint32_t BYTES = OFF_ABORT + 16;
+  static constexpr uint32_t OFF_CLAIM_CTR = OFF_ABORT + 16;   // u32; rank 0's counts the head's claims
+  static constexpr uint32_t OFF_CLAIMS = OFF_CLAIM_CTR + 16;  // [NCLAIM] s32: frame of job j, -1 = done
+  static constexpr uint32_t BYTES = OFF_CLAIMS + 4 * NCLAIM;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;              // base alignment slack
 
   // TMEM columns (each region 128 lanes)
@@ -198,19 +213,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): 8 values -> two 16-byte chunks.
-__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-  float h[8], l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const __nv_bfloat16 b = __float2bfloat16_rn(x[e]);
-    h[e] = __bfloat162float(b);
-    l[e] = x[e] - h[e];
-  }
-  hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
-                  pack_bf16x2(h[6], h[7]));
-  lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]),
-                  pack_bf16x2(l[6], l[7]));
+// Claims the next frame of the head: relaxed atomic add on the counter in the
+// shared memory of the cluster's rank 0 (cluster address). Returns the frame.
+__device__ __forceinline__ int claim_frame(uint32_t counter) {
+  uint32_t old;
+  asm volatile("atom.relaxed.cluster.shared::cluster.add.u32 %0, [%1], 1;"
+               : "=r"(old)
+               : "r"(counter)
+               : "memory");
+  return (int)old;
+}
+
+__device__ __forceinline__ int ld_shared_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// 8 floats -> one 16-byte chunk of bf16 (round to nearest even).
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
 }
 
 struct Ctl {
@@ -335,13 +358,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   const int T = p.T;
   const int ntile = p.ntile;
   const int nkv = p.nkv;
-  const int nown = (T > (int)rank) ? (T - (int)rank + P - 1) / P : 0;   // frames this CTA owns
 
   auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * i; };
   auto kv_slot = [&](int i) -> uint32_t { return sb + L::OFF_KV + i * L::KV_SLOT; };
   auto q_slot = [&](int i) -> uint32_t { return sb + L::OFF_Q + i * kTileBytes; };
   auto ac_slot = [&](int i) -> uint32_t { return sb + L::OFF_AC + i * L::AC_SLOT; };
   auto mch = [&](int i) -> uint32_t { return sb + L::OFF_MCH + i * L::M_BUF; };
+  // Frame of this CTA's job j (claimed by its K/V loader), or -1 past the last one.
+  auto claim_slot = [&](int j) -> uint32_t { return sb + L::OFF_CLAIMS + 4u * (j % L::NCLAIM); };
   // Output rows of this CTA, in every frame, and its Q tiles.
   const int r0 = (int)rank * p.chunk;
   const int r1 = min(p.S, r0 + p.chunk);
@@ -365,10 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_GB_FULL + i), 1);
       mbar_init(bar(L::B_GB_FREE + i), 4);
-      mbar_init(bar(L::B_MCH_FULL + i), 4);
-      mbar_init(bar(L::B_MCH_FREE + i), 1);
       mbar_init(bar(L::B_O_FULL + i), 1);
       mbar_init(bar(L::B_O_FREE + i), 4);
+    }
+    for (int i = 0; i < L::NM; ++i) {
+      mbar_init(bar(L::B_MCH_FULL + i), 4);
+      mbar_init(bar(L::B_MCH_FREE + i), 1);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(L::B_E1_STAGED + i), 4);
@@ -379,7 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
     for (int i = 0; i < 3; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
+    for (int i = 0; i < L::NCLAIM; ++i) mbar_init(bar(L::B_CLAIM + i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::OFF_CLAIM_CTR), "r"(0u) : "memory");
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -400,23 +428,45 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_ptr) : "memory");
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------ K/V loader (own frames)
-    // Tiles of the next own frame are prefetched into L2 while this one loads,
-    // so the loads below see L2 latency rather than loaded-HBM latency.
-    // Inputs are read once: evict them first, keeping L2 for the ring and prefetches.
+    // ------------------------------------------------ K/V loader (claims the frames to produce)
+    // The CTAs of a head claim the frames they produce from one counter in
+    // rank 0's shared memory, so a CTA that streams faster produces more of
+    // them. Each claim is made one frame ahead, and that frame's tiles are
+    // prefetched into L2 while the current one loads, so the loads below see L2
+    // latency rather than loaded-HBM latency. Inputs are read once: evict them
+    // first, keeping L2 for the ring and the prefetches.
     const uint64_t stream_pol = policy_evict_first();
-    for (int i = 0; i < nkv && (int)rank < T; ++i) {
-      tma_prefetch_3d(&p.tm_k, 0, i * kKvRows, bh * T + (int)rank);
-      tma_prefetch_3d(&p.tm_v, 0, i * kKvRows, bh * T + (int)rank);
+    const uint32_t counter = mapa(sb + L::OFF_CLAIM_CTR, 0);
+    auto prefetch_frame = [&](int f) {
+      for (int i = 0; i < nkv; ++i) {
+        tma_prefetch_3d(&p.tm_k, 0, i * kKvRows, bh * T + f);
+        tma_prefetch_3d(&p.tm_v, 0, i * kKvRows, bh * T + f);
+      }
+    };
+    int next = claim_frame(counter);
+    if (next < T) prefetch_frame(next);
+#ifdef GDN_TRACE
+    {
+      unsigned int sm;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+      GDN_TRACE_CTA(0, sm);
     }
+#endif
     int it = 0;
-    for (int j = 0; j < nown; ++j) {
-      const int f = (int)rank + j * P;
-      if (j + 1 < nown)
-        for (int i = 0; i < nkv; ++i) {
-          tma_prefetch_3d(&p.tm_k, 0, i * kKvRows, bh * T + f + P);
-          tma_prefetch_3d(&p.tm_v, 0, i * kKvRows, bh * T + f + P);
-        }
+    for (int j = 0;; ++j) {
+      const int f = next < T ? next : -1;
+      // Job j's frame for the MMA issuer, the A'/c warps and the publisher. They
+      // trail this loop by fewer than NCLAIM jobs, so the slot is free again.
+      asm volatile("st.shared.s32 [%0], %1;" ::"r"(claim_slot(j)), "r"(f) : "memory");
+      mbar_arrive(bar(L::B_CLAIM + j % L::NCLAIM));
+      if (f < 0) {
+        GDN_TRACE_CTA(2, globaltimer_ns());
+        GDN_TRACE_CTA(3, j);
+        break;
+      }
+      if (j == 2) GDN_TRACE_CTA(1, globaltimer_ns());
+      next = claim_frame(counter);
+      if (next < T) prefetch_frame(next);
       bool ok = true;
       for (int i = 0; i < nkv; ++i, ++it) {
         const int slot = it % L::NKV;
@@ -440,8 +490,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     // ------------------------------------------------ publisher of this CTA's frames
     // The fence and the release below wait for the producer warps' ring writes
     // to be performed; doing them here keeps the producer warps streaming.
-    for (int j = 0; j < nown; ++j) {
-      const int f = (int)rank + j * P;
+    for (int j = 0;; ++j) {
+      if (!wait_bar(bar(L::B_CLAIM + j % L::NCLAIM), (j / L::NCLAIM) & 1, ctl, kStProd)) break;
+      const int f = ld_shared_s32(claim_slot(j));
+      if (f < 0) break;
       if (!wait_bar(bar(L::B_E1_STAGED + (j & 3)), (j >> 2) & 1, ctl, kStProd)) break;
       GDN_TRACE_EV(20, j);
       __threadfence();
@@ -489,14 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          // A' M_{t-1} = A' M_hi + A' M_lo: A' is small next to the exact fp32
-          // gamma M term, so one bf16 copy of it suffices.
+          // A' M_{t-1} with both in bf16: the product is small next to the
+          // exact fp32 gamma M term it is added to, so its relative rounding
+          // error enters the state scaled down by |A'| / gamma.
           const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
-          const uint32_t mb = mch((t + 1) & 1) + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;   // M_{t-1}
+          const uint32_t mb = mch((t + L::NM - 1) % L::NM) + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
           const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
-          const uint64_t bL = smem_desc(mb + L::M_PART, L::MB_BLOCK, L::MB_SBO, 4);
           mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
-          mma_bf16(dt, aH, bL, id_chain, 1u);
         }
       }
       mma_commit(bar(L::B_CHAIN_DONE));
@@ -513,7 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     constexpr uint32_t id_gb = idesc_bf16(128, 64, 1, 1);      // [K V]^T and K, both MN-major
     int kvit = 0;
     bool ok = true;
-    for (int j = 0; j < nown && ok; ++j) {
+    for (int j = 0; ok; ++j) {
+      if (!wait_bar(bar(L::B_CLAIM + j % L::NCLAIM), (j / L::NCLAIM) & 1, ctl, kStMma)) break;
+      if (ld_shared_s32(claim_slot(j)) < 0) break;
       const int b = j & 1;
       if (!wait_bar(bar(L::B_GB_FREE + b), ((j >> 1) & 1) ^ 1, ctl, kStMma)) break;
       for (int i = 0; i < nkv; ++i, ++kvit) {
@@ -545,8 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     int qit = 0, on = 0;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
-      const int u = t & 1;
-      if (!wait_bar(bar(L::B_MCH_FULL + u), (t >> 1) & 1, ctl, kStMma)) break;
+      const int u = t % L::NM;
+      if (!wait_bar(bar(L::B_MCH_FULL + u), (t / L::NM) & 1, ctl, kStMma)) break;
       for (int i = 0; i < nq; ++i, ++qit, ++on) {
         const int slot = qit % L::NQ;
         const int ob = on & 1;
@@ -563,9 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t a = smem_desc(qt + kk * 32, 16, 1024, 2);
           const uint64_t bH = smem_desc(mo + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
-          const uint64_t bL = smem_desc(mo + L::M_PART + kk * 2 * L::MB_SBO, L::MB_BLOCK, L::MB_SBO, 4);
           mma_bf16(dO, a, bH, id_o, kk > 0 ? 1u : 0u);
-          mma_bf16(dO, a, bL, id_o, 1u);
         }
         mma_commit(bar(L::B_O_FULL + ob));
         if (i == 0 && t % P == (int)rank) GDN_TRACE_EV(15, t / P);
@@ -615,15 +666,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       m[jj] = p.state_in ? p.state_in[((size_t)bh * kD + row) * kD + 32 * hf + jj] : 0.f;
     auto store_state = [&](uint32_t buf) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 h, l;
-        split8(&m[8 * c], h, l);
-        const uint32_t off = hf * L::MB_BLOCK + swz_off(row, c, L::MB_RW, 2);
-        st_shared_v4(buf + off, h);
-        st_shared_v4(buf + L::M_PART + off, l);
-      }
+      for (int c = 0; c < 4; ++c)
+        st_shared_v4(buf + hf * L::MB_BLOCK + swz_off(row, c, L::MB_RW, 2), pack8(&m[8 * c]));
     };
-    store_state(mch(1));                       // M_{-1} = M_0, read by the first MMA
+    store_state(mch(L::NM - 1));               // M_{-1} = M_0, read by the first MMA
     fence_proxy_async_cta();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::B_M_READY));
@@ -637,13 +683,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       const int s = t % NAC;
       const bool acok = warp_wait(bar(L::B_AC_FULL + s), (t / NAC) & 1, ctl, kStChain);
       if (acok && lane == 0 && warp == 4) GDN_TRACE_EV(21, t);
-      // M_t goes to buffer t % 2, which held M_{t-2}: its read-out MMAs must be done.
+      // M_t goes to buffer t % NM, which held M_{t-NM}: its read-out MMAs must be done.
       uint32_t cd = 0;
       if (acok && lane == 0) cd = poll_bar(bar(L::B_CHAIN_DONE), t & 1, ctl, kStChain) ? 1u : 0u;
       cd = __shfl_sync(0xffffffffu, cd, 0);
       if (cd) mbar_test(bar(L::B_CHAIN_DONE), t & 1);    // acquire for every lane
       if (!acok || !cd ||
-          !warp_wait(bar(L::B_MCH_FREE + (t & 1)), ((t >> 1) & 1) ^ 1, ctl, kStMoEmpty)) {
+          !warp_wait(bar(L::B_MCH_FREE + t % L::NM), ((t / L::NM) & 1) ^ 1, ctl, kStMoEmpty)) {
         ok = false;
         break;
       }
@@ -669,14 +715,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         asm volatile("ld.shared.f32 %0, [%1];" : "=f"(cv) : "r"(ccol + jj * kD * 4) : "memory");
         m[jj] = fmaf(g, m[jj], __uint_as_float(d[jj])) + cv;
       }
-      store_state(mch(t & 1));
+      store_state(mch(t % L::NM));
       tc_fence_before();
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
         mbar_arrive(bar(L::B_AC_EMPTY + s));   // A'_t read by its MMA, c_t read here: slot free
-        mbar_arrive(bar(L::B_MCH_FULL + (t & 1)));   // M_t ready for the read-out
+        mbar_arrive(bar(L::B_MCH_FULL + t % L::NM));   // M_t ready for the read-out
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
     }
@@ -692,8 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const float* gam = p.gamma + (size_t)bh * T;
     const float* bet = p.beta + (size_t)bh * T;
     unsigned long long ring_seen = 0;            // lowest CTA progress last read (lane 0)
-    for (int j = 0; j < nown; ++j) {
-      const int f = (int)rank + j * P;
+    for (int j = 0;; ++j) {
+      if (!warp_wait(bar(L::B_CLAIM + j % L::NCLAIM), (j / L::NCLAIM) & 1, ctl, kStProd)) break;
+      const int f = ld_shared_s32(claim_slot(j));
+      if (f < 0) break;
       const int b = j & 1;
       const float g = __ldg(gam + f);
       const float be = __ldg(bet + f);
@@ -1135,6 +1183,10 @@ cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head) {
 extern "C" __attribute__((visibility("default"))) int gdn_trace_copy(void* dst, size_t bytes) {
   const size_t n = sizeof(g_trace) < bytes ? sizeof(g_trace) : bytes;
   return cudaMemcpyFromSymbol(dst, g_trace, n) == cudaSuccess ? (int)n : -1;
+}
+extern "C" __attribute__((visibility("default"))) int gdn_trace_cta_copy(void* dst, size_t bytes) {
+  const size_t n = sizeof(g_trace_cta) < bytes ? sizeof(g_trace_cta) : bytes;
+  return cudaMemcpyFromSymbol(dst, g_trace_cta, n) == cudaSuccess ? (int)n : -1;
 }
 extern "C" __attribute__((visibility("default"))) int gdn_trace_heads_copy(void* dst, size_t bytes) {
   const size_t n = sizeof(g_trace_heads) < bytes ? sizeof(g_trace_heads) : bytes;
