@@ -19,6 +19,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -67,13 +68,22 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments or blank lines, so that documentation
+    edits do not count as kernel changes."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """SHA-256 of the kernel sources' code (comments removed)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "frame_wise_gated_scan_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

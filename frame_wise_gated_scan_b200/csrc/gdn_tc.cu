@@ -12,21 +12,28 @@
 // D x D x D product A' M. The read-out O = Q M' follows behind it.
 //
 // Work split. One thread-block cluster of P CTAs per head (P = 1, 2 or 4):
-//  * frames are dealt round-robin: CTA r owns frames r, r+P, ...; for its
-//    frames it streams K, V, Q (TMA, 128-row tiles, 128-byte swizzle), forms
-//    [G; (K^T V)^T] = [K V]^T K on the tensor cores, turns it into A' (bf16
-//    hi + lo) and c, and writes them into every CTA's shared memory;
-//  * the value columns of the state never mix, so CTA r runs the recurrence
-//    for its NC = 64/P state columns on every frame: its fp32 slice of M
-//    stays in registers across all T frames, and its bf16 hi/lo copy is the
-//    MMA operand of the next frame;
-//  * each CTA sends its slice of M_t to the owner of frame t, which computes
-//    O_t = Q_t M_t (M in bf16 hi + lo, two MMAs) and stores it.
-// Warp roles (512 threads): warp 0 K/V loader (lane 0) and ring publisher
-// (lane 16); warp 1 Q loader (lane 0) and [K V]^T K MMA issuer (lane 16); warp 2
-// recurrence MMA issuer (lane 0, and TMEM allocation); warp 3 ring loader
-// (lane 0) and read-out MMA issuer (lane 16); warps 4-7 recurrence epilogue;
-// 8-11 A'/c epilogue; 12-15 output epilogue.
+//  * production: the CTAs of a head claim frames from a counter in rank 0's
+//    shared memory (so a faster SM produces more of them). For a claimed
+//    frame a CTA streams K and V (TMA, 64-row tiles, 128-byte swizzle), forms
+//    [G; (K^T V)^T] = [K V]^T K on the tensor cores, and turns it into A'
+//    (bf16) and c^T (fp32);
+//  * with P > 1 those operands go to a ring in global memory that stays in L2
+//    (16 frames per head), published with a release flag; every CTA of the
+//    head, the producer included, bulk-loads every frame from it in frame
+//    order. With P = 1 they are written straight into shared memory;
+//  * every CTA runs the whole recurrence: the fp32 state M stays in the
+//    registers of four warps across all T frames (gamma M is added in exact
+//    fp32), and its bf16 copy in shared memory is the operand of the next
+//    frame's MMA A' M;
+//  * CTA r reads out its own block of rows [r*chunk, (r+1)*chunk) of every
+//    frame, O_t = Q_t M_t, from its own copy of M_t (four bf16 buffers, so the
+//    read-out may trail the recurrence by up to four frames), and stores it
+//    with TMA.
+// Warp roles (512 threads): warp 0 K/V loader and frame claims (lane 0) and
+// ring publisher (lane 16); warp 1 Q loader (lane 0) and [K V]^T K MMA issuer
+// (lane 16); warp 2 recurrence MMA issuer (lane 0, and TMEM allocation); warp 3
+// ring loader (lane 0) and read-out MMA issuer (lane 16); warps 4-7 recurrence
+// epilogue; 8-11 A'/c epilogue; 12-15 output epilogue.
 //
 // Every wait is bounded (kTimeoutNs). A wait that runs out sets the device
 // status word and an abort flag in every CTA of the cluster; the other roles
@@ -185,7 +192,8 @@ struct TcParams {
   uint16_t* out;           // bf16 bit patterns
   unsigned int* status;
   // Transition operands shared by the CTAs of a head (P > 1), per head:
-  // kRing frames of [A' hi | A' lo | c], their ready flags and per-CTA progress.
+  // kRing frames of [A' (bf16, K-major, swizzled) | c^T (fp32)], their ready
+  // flags and per-CTA progress.
   uint8_t* ring;                     // [heads][kRing][AC_BYTES]
   unsigned long long* ring_flag;     // [heads][kRing]: frame + 1 once published
   unsigned long long* ring_loaded;   // [heads][P]: frames loaded by each CTA
