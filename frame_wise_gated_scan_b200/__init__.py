@@ -5,8 +5,9 @@ frame_scan_noalloc, for callers that must not allocate device memory) from
 frame_wise_gated_scan_b200.gdn; the library is built in-tree by
 frame_wise_gated_scan_b200.build.
 """
-from .gdn import (GdnError, KERNEL_SIMT, KERNEL_TC, device_status, frame_scan, frame_scan_host,
+from .gdn import (FLAG_NO_DELTA, GdnError, KERNEL_SIMT, KERNEL_TC, device_status, frame_scan,
+                  frame_scan_host,
                   frame_scan_noalloc, frame_step, plan, version)
 
-__all__ = ["GdnError", "KERNEL_SIMT", "KERNEL_TC", "device_status", "frame_scan",
+__all__ = ["FLAG_NO_DELTA", "GdnError", "KERNEL_SIMT", "KERNEL_TC", "device_status", "frame_scan",
            "frame_scan_host", "frame_scan_noalloc", "frame_step", "plan", "version"]

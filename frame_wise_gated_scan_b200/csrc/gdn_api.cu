@@ -51,9 +51,10 @@ int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
 
 int run(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
         const float* state_in, float* state_out, void* out, int B, int H, int T, int S, int D,
-        void* stream, int elt_bytes, bool noalloc = false) {
+        void* stream, int elt_bytes, bool noalloc = false, unsigned int flags = 0) {
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
+  if (flags & ~GDN_FLAG_NO_DELTA) return GDN_ERR_FLAGS;
   if (noalloc && (long long)B * H > GDN_NOALLOC_MAX_HEADS) return GDN_ERR_SCRATCH;
   if (!q || !k || !v || !gamma || !beta || !out) return GDN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
@@ -83,6 +84,7 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   p.S = S;
   p.D = D;
   p.key_scale = (float)(1.0 / sqrt((double)D * (double)S));
+  p.delta = (flags & GDN_FLAG_NO_DELTA) == 0;
   p.stream = static_cast<cudaStream_t>(stream);
 
   cudaError_t err;
@@ -133,6 +135,30 @@ int gdn_frame_step_f32(const float* q, const float* k, const float* v, const flo
   return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 4);
 }
 
+int gdn_frame_scan_ex(const void* q, const void* k, const void* v, const float* gamma,
+                      const float* beta, const float* state_in, float* state_out, void* out, int B,
+                      int H, int T, int S, int D, unsigned int flags, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 2, false, flags);
+}
+
+int gdn_frame_step_ex(const void* q, const void* k, const void* v, const float* gamma,
+                      const float* beta, const float* state_in, float* state_out, void* out, int B,
+                      int H, int S, int D, unsigned int flags, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 2, false, flags);
+}
+
+int gdn_frame_scan_f32_ex(const float* q, const float* k, const float* v, const float* gamma,
+                          const float* beta, const float* state_in, float* state_out, float* out,
+                          int B, int H, int T, int S, int D, unsigned int flags, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, T, S, D, stream, 4, false, flags);
+}
+
+int gdn_frame_step_f32_ex(const float* q, const float* k, const float* v, const float* gamma,
+                          const float* beta, const float* state_in, float* state_out, float* out,
+                          int B, int H, int S, int D, unsigned int flags, void* stream) {
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 4, false, flags);
+}
+
 int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head) {
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
@@ -160,6 +186,7 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_ALIAS: return "out overlaps an input or a state buffer";
     case GDN_ERR_SCRATCH:
       return "B * H exceeds GDN_NOALLOC_MAX_HEADS (32), the fixed scratch of gdn_frame_scan_noalloc";
+    case GDN_ERR_FLAGS: return "flags holds bits other than GDN_FLAG_NO_DELTA";
     default: return "unknown gdn_status";
   }
 }

@@ -18,6 +18,7 @@ struct Problem {
   void* out;
   int B, H, T, S, D;
   float key_scale;         // 1/sqrt(D*S), rounded once from double
+  bool delta;              // delta-rule correction on (false: GDN_FLAG_NO_DELTA, R = V)
   cudaStream_t stream;
 };
 

@@ -4,7 +4,8 @@
 // section "A Arquitetura", item "1. Atencao Linear Hibrida com Gated DeltaNet":
 // per frame W = (sK)M, R = V - gamma W, M <- gamma M + beta (sK)^T R, O = Q M,
 // in that order and in fp32. They serve the fp32-input calls and the bf16
-// calls the tensor-core kernel does not take.
+// calls the tensor-core kernel does not take. Without the delta rule
+// (GDN_FLAG_NO_DELTA) the residual is V itself and W is not formed.
 //
 // Decomposition: the value columns of M never mix (column j of W, R, the
 // update and O only involves column j of M and V), so each CTA owns one
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(kThreads)
 gdn_simt_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k,
                 const Elt* __restrict__ v, const float* __restrict__ gamma,
                 const float* __restrict__ beta, const float* state_in, float* state_out,
-                Elt* __restrict__ out, int T, int S, float s) {
+                Elt* __restrict__ out, int T, int S, float s, bool delta) {
   constexpr int kAcc = D * kCB / kThreads;   // K^T R elements per thread
   static_assert(kAcc * kThreads == D * kCB, "D must be a multiple of 16");
   __shared__ float Ms[D][kCB];               // state columns [j0, j0+16)
@@ -78,10 +79,14 @@ gdn_simt_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k,
       __syncthreads();
       for (int e = tid; e < kTS * kCB; e += kThreads) {
         const int r = e / kCB, j = e % kCB;
-        float w = 0.f;
+        if (delta) {
+          float w = 0.f;
 #pragma unroll 8
-        for (int d = 0; d < D; ++d) w = fmaf(Xs[r][d], Ms[d][j], w);
-        Rs[r][j] = Vs[r][j] - g * w;
+          for (int d = 0; d < D; ++d) w = fmaf(Xs[r][d], Ms[d][j], w);
+          Rs[r][j] = Vs[r][j] - g * w;
+        } else {
+          Rs[r][j] = Vs[r][j];
+        }
       }
       __syncthreads();
 #pragma unroll
@@ -143,15 +148,15 @@ cudaError_t launch(const Problem& p) {
   switch (p.D) {
     case 32:
       gdn_simt_kernel<Elt, 32><<<grid, kThreads, 0, p.stream>>>(
-          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale);
+          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale, p.delta);
       break;
     case 64:
       gdn_simt_kernel<Elt, 64><<<grid, kThreads, 0, p.stream>>>(
-          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale);
+          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale, p.delta);
       break;
     case 128:
       gdn_simt_kernel<Elt, 128><<<grid, kThreads, 0, p.stream>>>(
-          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale);
+          q, k, v, p.gamma, p.beta, p.state_in, p.state_out, out, p.T, p.S, p.key_scale, p.delta);
       break;
     default:
       return cudaErrorInvalidValue;

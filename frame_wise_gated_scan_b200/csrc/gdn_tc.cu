@@ -204,6 +204,7 @@ struct TcParams {
   int chunk;        // output rows per CTA (multiple of 16); CTA r owns [r*chunk, (r+1)*chunk)
   float s;     // key scale 1/sqrt(D*S)
   float s2;    // its square
+  float delta; // 1: delta rule; 0: GDN_FLAG_NO_DELTA, so A' = 0 and M' = gamma M + c
 };
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
@@ -772,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       // A' rows are packed in place: chunk c (8 values) becomes 4 bf16x2 words in
       // v[8c..8c+3].
       if (lrow < kD) {
-        const float coef = -g * be * p.s2;       // A' = -gamma beta s^2 G
+        const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 G (0 without delta)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float x[8];
@@ -1090,6 +1091,7 @@ cudaError_t launch_p(const Problem& pr, uint8_t* fixed_scratch) {
   p.s = pr.key_scale;
   const double sd = 1.0 / ((double)kD * (double)pr.S);
   p.s2 = (float)sd;
+  p.delta = pr.delta ? 1.f : 0.f;
 
   // Ring of transition operands shared by the CTAs of each head (P > 1):
   // stream-ordered scratch, released right after the launch on the same stream.

@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
 
 KERNEL_SIMT = 1
 KERNEL_TC = 2
+FLAG_NO_DELTA = 1     # GDN_FLAG_NO_DELTA: R = V, the decayed cumulative (block KV cache) form
 
 _lib = None
 
@@ -51,6 +52,14 @@ def lib() -> ctypes.CDLL:
         for name, args in (("gdn_frame_scan", scan_args), ("gdn_frame_scan_f32", scan_args),
                            ("gdn_frame_scan_noalloc", scan_args),
                            ("gdn_frame_step", step_args), ("gdn_frame_step_f32", step_args)):
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = i
+        u = ctypes.c_uint
+        for name, args in (("gdn_frame_scan_ex", scan_args[:-1] + [u, vp]),
+                           ("gdn_frame_scan_f32_ex", scan_args[:-1] + [u, vp]),
+                           ("gdn_frame_step_ex", step_args[:-1] + [u, vp]),
+                           ("gdn_frame_step_f32_ex", step_args[:-1] + [u, vp])):
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = i
@@ -108,7 +117,7 @@ def _check(t, name, dtype, shape, device):
 
 
 def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state,
-          noalloc=False):
+          noalloc=False, flags=0):
     if q.dim() != (4 if step else 5):
         raise ValueError("q must be [B,H,S,D] for a step, [B,H,T,S,D] for a scan")
     device = q.device
@@ -143,8 +152,17 @@ def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state
             _ptr(state_out), _ptr(out), B, H]
     if not step:
         args.append(T)
-    args += [S, D, _stream_handle(device)]
-    if noalloc:
+    args += [S, D]
+    if flags:
+        args.append(flags)
+    args.append(_stream_handle(device))
+    bf16 = dt == torch.bfloat16
+    if flags:
+        if step:
+            fn = L.gdn_frame_step_ex if bf16 else L.gdn_frame_step_f32_ex
+        else:
+            fn = L.gdn_frame_scan_ex if bf16 else L.gdn_frame_scan_f32_ex
+    elif noalloc:
         fn = L.gdn_frame_scan_noalloc
     elif step:
         fn = L.gdn_frame_step if dt == torch.bfloat16 else L.gdn_frame_step_f32
@@ -158,12 +176,14 @@ def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state
 
 
 def frame_scan(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
-               want_state=True):
+               want_state=True, delta=True):
     """T frames per head. q, k, v: [B,H,T,S,D] bf16 or fp32 CUDA tensors;
     gamma, beta: [B,H,T] fp32; state_in: [B,H,D,D] fp32 or None (zero).
+    delta=False drops the delta-rule correction (GDN_FLAG_NO_DELTA: R = V).
     Returns (out, state_out); state_out is None if want_state is False and
     none was given."""
-    return _call(False, q, k, v, gamma, beta, state_in, out, state_out, want_state)
+    return _call(False, q, k, v, gamma, beta, state_in, out, state_out, want_state,
+                 flags=0 if delta else FLAG_NO_DELTA)
 
 
 def frame_scan_noalloc(q, k, v, gamma, beta, state_in=None, *, out, state_out=None):
@@ -180,10 +200,12 @@ def frame_scan_noalloc(q, k, v, gamma, beta, state_in=None, *, out, state_out=No
 
 
 def frame_step(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
-               want_state=True):
+               want_state=True, delta=True):
     """One frame per head (chunk-causal rollout). q, k, v: [B,H,S,D];
-    gamma, beta: [B,H]. state_out may be state_in (in-place carry)."""
-    return _call(True, q, k, v, gamma, beta, state_in, out, state_out, want_state)
+    gamma, beta: [B,H]. state_out may be state_in (in-place carry).
+    delta=False as in frame_scan."""
+    return _call(True, q, k, v, gamma, beta, state_in, out, state_out, want_state,
+                 flags=0 if delta else FLAG_NO_DELTA)
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,

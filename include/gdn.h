@@ -70,7 +70,8 @@ typedef enum gdn_status {
   GDN_ERR_CUDA = -5,            /* a CUDA runtime or driver call failed */
   GDN_ERR_TIMEOUT = -6,         /* a device-side wait ran out (from gdn_device_status) */
   GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
-  GDN_ERR_SCRATCH = -8          /* B * H > GDN_NOALLOC_MAX_HEADS (gdn_frame_scan_noalloc) */
+  GDN_ERR_SCRATCH = -8,         /* B * H > GDN_NOALLOC_MAX_HEADS (gdn_frame_scan_noalloc) */
+  GDN_ERR_FLAGS = -9            /* unknown bits in `flags` (the _ex calls) */
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
@@ -140,6 +141,34 @@ GDN_API int gdn_frame_step_f32(const float* q, const float* k, const float* v,
                        const float* gamma, const float* beta,
                        const float* state_in, float* state_out, float* out,
                        int B, int H, int S, int D, void* stream);
+
+/* Variants with a `flags` word (0 gives exactly the calls above).
+ *
+ * GDN_FLAG_NO_DELTA: the update without the delta-rule correction, R = V_t:
+ *     M_t = gamma_t M_{t-1} + beta_t (s K_t)^T V_t,   O_t = Q_t M_t.
+ * This is the decayed cumulative state of block-causal linear attention, the
+ * block KV cache of SANA-Video ("SANA-Video" ICLR 2026 oral transcript,
+ * shadowingenglish.com, the part on block causal linear attention). With
+ * gamma = beta = 1 it is plain cumulative linear attention over the frames
+ * so far. Same kernels, layouts and precision as the delta-rule calls.
+ * Any other bit returns GDN_ERR_FLAGS. */
+#define GDN_FLAG_NO_DELTA 1u
+GDN_API int gdn_frame_scan_ex(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int T, int S, int D, unsigned int flags, void* stream);
+GDN_API int gdn_frame_step_ex(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int S, int D, unsigned int flags, void* stream);
+GDN_API int gdn_frame_scan_f32_ex(const float* q, const float* k, const float* v,
+                       const float* gamma, const float* beta,
+                       const float* state_in, float* state_out, float* out,
+                       int B, int H, int T, int S, int D, unsigned int flags, void* stream);
+GDN_API int gdn_frame_step_f32_ex(const float* q, const float* k, const float* v,
+                       const float* gamma, const float* beta,
+                       const float* state_in, float* state_out, float* out,
+                       int B, int H, int S, int D, unsigned int flags, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
  * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head

@@ -37,9 +37,10 @@ def to_np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def oracle_head(wl: inputs.Workload, b: int, h: int, T: int | None = None, state_in=None):
+def oracle_head(wl: inputs.Workload, b: int, h: int, T: int | None = None, state_in=None,
+                delta: bool = True):
     q, k, v, g, be = inputs.head(wl, b, h, T)
-    return gdn_scan_ref(q, k, v, g, be, state_in=state_in)
+    return gdn_scan_ref(q, k, v, g, be, state_in=state_in, delta=delta)
 
 
 def assert_close(out, ref_out, state, ref_state, tol, what=""):

@@ -19,7 +19,9 @@ def L():
 def test_every_declared_symbol_is_exported(L):
     names = gdn.header_symbols()
     assert set(names) >= {"gdn_frame_scan", "gdn_frame_step", "gdn_frame_scan_f32",
-                          "gdn_frame_step_f32", "gdn_frame_scan_noalloc", "gdn_plan",
+                          "gdn_frame_step_f32", "gdn_frame_scan_noalloc", "gdn_frame_scan_ex",
+                          "gdn_frame_step_ex", "gdn_frame_scan_f32_ex", "gdn_frame_step_f32_ex",
+                          "gdn_plan",
                           "gdn_device_status",
                           "gdn_status_string", "gdn_version"}
     out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
@@ -34,7 +36,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strings(L):
     assert gdn.version() == 10000
-    for st in range(-8, 1):
+    for st in range(-9, 1):
         s = gdn.status_string(st)
         assert s and s != "unknown gdn_status"
     assert gdn.status_string(-99) == "unknown gdn_status"
@@ -74,6 +76,20 @@ def test_step_and_f32_entry_points_validate(L):
                             p(0x6000), 1, 1, 8, 64, None) == -1
     assert L.gdn_frame_step_f32(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), None,
                                 None, p(0x7000), 1, 1, 8, 96, None) == -3
+
+
+def test_flags_are_checked_on_the_host(L):
+    p = ctypes.c_void_p
+    args = [p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), None, None, p(0x100000)]
+    assert L.gdn_frame_scan_ex(*args, 1, 2, 3, 64, 64, 2, None) == -9      # unknown bit
+    assert L.gdn_frame_scan_ex(*args, 1, 2, 3, 64, 64, 0x80000000, None) == -9
+    assert L.gdn_frame_step_ex(*args, 1, 2, 64, 64, 4, None) == -9
+    assert L.gdn_frame_scan_f32_ex(*args, 1, 2, 3, 64, 64, 3, None) == -9
+    assert L.gdn_frame_step_f32_ex(*args, 1, 2, 64, 64, 8, None) == -9
+    # the ordinary checks still come first
+    assert L.gdn_frame_scan_ex(None, *args[1:], 1, 2, 3, 64, 64, 1, None) == -1
+    assert L.gdn_frame_scan_ex(*args, 1, 2, 3, 64, 48, 1, None) == -3
+    assert "GDN_FLAG_NO_DELTA" in gdn.status_string(-9)
 
 
 def test_plan_is_host_logic(L):

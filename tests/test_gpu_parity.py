@@ -23,17 +23,17 @@ def workload_on_device(name, T=None):
     return _cache[key]
 
 
-def _scan_and_compare(wl, heads=None, T=None, tol=None, state_in=None):
+def _scan_and_compare(wl, heads=None, T=None, tol=None, state_in=None, delta=True):
     q, k, v, g, be = device_workload(wl, T)
     st_dev = None if state_in is None else torch.from_numpy(state_in).cuda()
-    out, st = gdn.frame_scan(q, k, v, g, be, st_dev)
+    out, st = gdn.frame_scan(q, k, v, g, be, st_dev, delta=delta)
     torch.cuda.synchronize()
     assert gdn.device_status() == 0
     tol = tol or (TOL_F32 if wl.dtype == "f32" else TOL_BF16)
     heads = heads or [(b, h) for b in range(wl.B) for h in range(wl.H)]
     worst = 0.0
     for b, h in heads:
-        ro, rs = oracle_head(wl, b, h, T, None if state_in is None else state_in[b, h])
+        ro, rs = oracle_head(wl, b, h, T, None if state_in is None else state_in[b, h], delta)
         e, _ = assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, tol, f"{wl.name} b{b} h{h}")
         worst = max(worst, e)
     return worst
@@ -175,3 +175,46 @@ def test_host_buffers_end_to_end():
     hq, hk, hv, hg, hb = (x.cpu().pin_memory() for x in (q, k, v, g, be))
     o, s = gdn.frame_scan_host(hq, hk, hv, hg, hb)
     assert torch.equal(o, ref_o.cpu()) and torch.equal(s, ref_s.cpu())
+
+
+# ---- GDN_FLAG_NO_DELTA: R = V, the decayed cumulative (block KV cache) form ----
+
+@pytest.mark.parametrize("ctas", ["1", "2", "4"])
+def test_bf16_no_delta_tensor_core(monkeypatch, ctas):
+    monkeypatch.setenv("GDN_TC_CTAS", ctas)
+    wl = inputs.Workload(f"nodelta_tc{ctas}", 1, 3, 64, 19, 200, "bf16", 500 + int(ctas), "l2",
+                         "rollout")
+    assert gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D) == (gdn.KERNEL_TC, int(ctas))
+    _scan_and_compare(wl, state_in=inputs.state(wl, scale=0.5), delta=False)
+
+
+@pytest.mark.parametrize("D", [32, 128])
+def test_bf16_no_delta_cuda_cores(D):
+    wl = inputs.Workload(f"nodelta_d{D}", 1, 2, D, 5, 130, "bf16", 510 + D, "gauss", "tiny")
+    _scan_and_compare(wl, state_in=inputs.state(wl, scale=0.5), delta=False)
+
+
+def test_fp32_no_delta():
+    wl = inputs.WORKLOADS["tiny"]
+    _scan_and_compare(wl, state_in=inputs.state(wl), delta=False)
+
+
+def test_no_delta_differs_from_delta_and_step_chain_equals_scan():
+    """The flag changes the result, and a chain of no-delta steps equals the
+    no-delta scan bit for bit (same kernel, one frame per call)."""
+    wl = inputs.Workload("nodelta_chain", 1, 2, 64, 6, 300, "bf16", 520, "l2", "rollout")
+    q, k, v, g, be = device_workload(wl)
+    out_d, st_d = gdn.frame_scan(q, k, v, g, be)
+    out_n, st_n = gdn.frame_scan(q, k, v, g, be, delta=False)
+    assert not torch.equal(st_d, st_n)
+    state = torch.zeros((wl.B, wl.H, wl.D, wl.D), device="cuda")
+    for t in range(wl.T):
+        o_t, _ = gdn.frame_step(q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                v[:, :, t].contiguous(), g[:, :, t].contiguous(),
+                                be[:, :, t].contiguous(), state, state_out=state, delta=False)
+        e_o = float((o_t.float() - out_n[:, :, t].float()).norm() / out_n[:, :, t].float().norm())
+        assert e_o <= 1e-2, f"frame {t}: no-delta step output vs scan {e_o:.3e}"
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    e = float((state - st_n).norm() / st_n.norm())
+    assert e <= 1e-6, f"no-delta step chain vs scan: {e:.3e}"
