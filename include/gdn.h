@@ -75,8 +75,14 @@ typedef enum gdn_status {
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
- * Arithmetic: fp32 accumulation on tcgen05 tensor cores, fp32 state kept on
- * chip across all T frames, out rounded to bf16 (round to nearest even). */
+ * Arithmetic (D = 64, tensor-core kernel): K^T K and K^T V accumulate in fp32
+ * on tcgen05 tensor cores; the state M is kept in fp32 on chip across all T
+ * frames and updated as M <- gamma M + A' M + c in fp32 registers, where the
+ * product A' M (A' = -gamma beta s^2 K^T K) and the read-out Q M take M and
+ * A' rounded to bf16 with fp32 accumulation; out is rounded to bf16 (round
+ * to nearest even). D = 32 and 128 run the update in fp32 on CUDA cores.
+ * On the seeded rollout workload the per-frame relative error against a
+ * float64 reference is about 2.4e-3 for out and 2e-6 for the final state. */
 GDN_API int gdn_frame_scan(const void* q, const void* k, const void* v,
                    const float* gamma, const float* beta,
                    const float* state_in, float* state_out, void* out,
