@@ -255,7 +255,7 @@ def main():
         return
     import torch
     import torch.distributed as dist
-    from frame_wise_gated_scan_b200 import gdn
+    from frame_wise_gated_scan_b200 import gdn, multi
 
     rank, world, local = dist_env()
     if world > 1:
@@ -300,13 +300,10 @@ def main():
     launch_ms = [a.elapsed_time(b) for a, b in launch_ev]
     if gdn.device_status() != 0:
         raise RuntimeError("a device-side wait ran out during the timed steps")
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = multi.max_over_ranks(elapsed_ms, device)
 
     units = wl.heads * wl.T
-    value = units * args.steps * world / (max_ms / 1e3)
+    value = multi.whole_job_rate(units, args.steps, world, max_ms)
     mean_launch_s = statistics.mean(launch_ms) / 1e3
     alg_bytes = inputs.algorithmic_bytes(wl)
     achieved = alg_bytes / mean_launch_s / 1e9
@@ -331,12 +328,10 @@ def main():
                                 state_host=st_h)
         e1.record(stream)
         torch.cuda.synchronize(device)
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = multi.max_over_ranks(e0.elapsed_time(e1), device)
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb))
         d2h = out_h.numel() * out_h.element_size() + st_h.numel() * 4
-        e2e = {"value": units * args.e2e_steps * world / (float(te.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": multi.whole_job_rate(units, args.e2e_steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": args.e2e_steps}
 
