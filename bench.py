@@ -208,7 +208,6 @@ def run_reference(args, wl):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    cb_seconds = max(1.0, min(args.cpu_seconds, 60.0))
     # each step: the oracle over one head for a bounded number of frames
     T = min(wl.T, 24)
     from oracle import gdn_scan_ref
@@ -239,7 +238,6 @@ def run_reference(args, wl):
                          "sample": f"{args.steps} steps of {T} frames of one head (S={wl.S}, D={wl.D})"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    del cb_seconds
     print(json.dumps(line), flush=True)
 
 
