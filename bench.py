@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--frames", type=int, default=0,
                     help="run only the first N frames of the workload (profiling captures)")
+    ap.add_argument("--step-calls", type=int, default=200,
+                    help="gdn_frame_step calls timed one by one for the step latency (0: skip)")
     return ap.parse_args()
 
 
@@ -307,6 +309,44 @@ def main():
     achieved = alg_bytes / mean_launch_s / 1e9
     peak, peak_kind = measured_peaks()
 
+    # Chunk-causal rollout, one gdn_frame_step per frame with the state carried in
+    # place (the "step" workload): per-call latency, after the timed region.
+    step_lat = None
+    if args.step_calls > 0:
+        n = min(args.step_calls, wl.T)
+        frames = [tuple(x[:, :, t].contiguous() for x in (q, k, v, g, be)) for t in range(n)]
+        o_step = torch.empty((wl.B, wl.H, wl.S, wl.D), dtype=q.dtype, device=device)
+        s_step = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
+        step_kern, step_ctas = gdn.plan(wl.B, wl.H, 1, wl.S, wl.D)
+        for t in range(min(3, n)):
+            gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
+        torch.cuda.synchronize(device)
+        s_step.zero_()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        host_us = []
+        for t in range(n):
+            h0 = time.perf_counter()
+            evs[t][0].record(stream)
+            gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
+            evs[t][1].record(stream)
+            torch.cuda.synchronize(device)
+            host_us.append((time.perf_counter() - h0) * 1e6)
+        if gdn.device_status() != 0:
+            raise RuntimeError("a device-side wait ran out during the step calls")
+        dev_us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+        host_us.sort()
+        pct = lambda xs, p: xs[min(len(xs) - 1, int(round(p / 100 * (len(xs) - 1))))]
+        step_lat = {"calls": n, "unit": "us",
+                    "device_p50": pct(dev_us, 50), "device_p99": pct(dev_us, 99),
+                    "host_p50": pct(host_us, 50), "host_p99": pct(host_us, 99),
+                    # q, k, v read, out written, gates, the state read and written
+                    "bytes_per_call": inputs.algorithmic_bytes(wl, 1) + wl.heads * wl.D * wl.D * 4,
+                    "kernel": {1: "simt", 2: "tcgen05"}[step_kern], "ctas_per_head": step_ctas,
+                    "how": "device: CUDA events around each call on its stream; host: call "
+                           "plus synchronize, wall clock"}
+        del frames
+
     # End to end through the public API on pinned host buffers.
     e2e = None
     if args.e2e_steps > 0:
@@ -357,6 +397,7 @@ def main():
                      "algorithmic_bytes_per_launch": alg_bytes},
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "step_latency": step_lat,
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
