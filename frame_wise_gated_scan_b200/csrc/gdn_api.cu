@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "gdn.h"
 #include "gdn_internal.h"
 
@@ -20,13 +22,16 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 // Kernel override for debugging: GDN_IMPL=simt forces the CUDA-core kernel.
+// Read once per process.
 int forced_kernel() {
-  static int cached = -1;
-  if (cached < 0) {
+  static std::atomic<int> cached{-1};
+  int v = cached.load(std::memory_order_relaxed);
+  if (v < 0) {
     const char* e = getenv("GDN_IMPL");
-    cached = (e && strcmp(e, "simt") == 0) ? GDN_KERNEL_SIMT : 0;
+    v = (e && strcmp(e, "simt") == 0) ? GDN_KERNEL_SIMT : 0;
+    cached.store(v, std::memory_order_relaxed);
   }
-  return cached;
+  return v;
 }
 
 int check_sizes(int B, int H, int T, int S, int D) {

@@ -44,6 +44,7 @@
 #include <stdlib.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "gdn.h"
 #include "gdn_internal.h"
@@ -365,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   const uint32_t rank = cluster_ctarank();
   const int bh = blockIdx.x / P;
   const int T = p.T;
-  const int ntile = p.ntile;
   const int nkv = p.nkv;
 
   auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * i; };
@@ -952,18 +952,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process.
 EncodeTiledFn encode_fn() {
+  static std::once_flag once;
   static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  std::call_once(once, [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+  });
   return fn;
 }
 
@@ -986,30 +986,35 @@ const void* kernel_ptr() {
   return reinterpret_cast<const void*>(&gdn_tc_kernel<P>);
 }
 
+// Raises the kernel's dynamic shared-memory limit. The attribute belongs to the
+// kernel on each device, so it is set once per device (concurrent first calls
+// both set it, which is harmless).
 template <int P>
 cudaError_t prepare() {
-  static bool done = false;
-  static cudaError_t err = cudaSuccess;
-  if (!done) {
-    err = cudaFuncSetAttribute(kernel_ptr<P>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)Layout<P>::SMEM_ALLOC);
-    done = true;
-  }
-  return err;
+  static std::atomic<bool> done[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel_ptr<P>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Layout<P>::SMEM_ALLOC);
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 // Clusters of P CTAs that can be resident at once on the current device, or
 // -1 if there is no usable device (host-only planning). Cached per device.
 template <int P>
 int resident_clusters() {
-  static int cache[64];
-  static bool have[64] = {};
+  static std::atomic<int> cache[64];            // 0: not yet known; else the count + 2
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return -1;
   }
-  if (have[dev]) return cache[dev];
+  const int known = cache[dev].load(std::memory_order_acquire);
+  if (known != 0) return known - 2;
   int n = -1;
   if (prepare<P>() == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -1026,21 +1031,23 @@ int resident_clusters() {
     if (cudaOccupancyMaxActiveClusters(&n, gdn_tc_kernel<P>, &cfg) != cudaSuccess) n = -1;
   }
   cudaGetLastError();
-  cache[dev] = n;
-  have[dev] = true;
+  cache[dev].store(n + 2, std::memory_order_release);
   return n;
 }
 
+// Address of the device status word on the current device, looked up once per device.
 unsigned int* status_word() {
-  static unsigned int* cache[64] = {};
+  static std::atomic<unsigned int*> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
+  unsigned int* a = cache[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_tc_status) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<unsigned int*>(ptr);
+    a = static_cast<unsigned int*>(ptr);
+    cache[dev].store(a, std::memory_order_release);
   }
-  return cache[dev];
+  return a;
 }
 
 // Address of g_noalloc_scratch on the current device. cudaGetSymbolAddress
