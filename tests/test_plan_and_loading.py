@@ -1,0 +1,64 @@
+"""Host logic that needs no GPU: which kernel and cluster size a call gets, and
+that the product path fails loudly, with no fallback, when the library is
+missing."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+from frame_wise_gated_scan_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+TC, SIMT = gdn.KERNEL_TC, gdn.KERNEL_SIMT
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="with a device the thresholds come from its cluster occupancy")
+def test_plan_without_a_device(monkeypatch):
+    monkeypatch.delenv("GDN_TC_CTAS", raising=False)
+    # 148 SMs assumed: 37 clusters of 4, 74 of 2 fit at once
+    assert gdn.plan(1, 32, 961, 880, 64) == (TC, 4)
+    assert gdn.plan(1, 37, 2, 64, 64) == (TC, 4)
+    assert gdn.plan(1, 38, 2, 64, 64) == (TC, 2)
+    assert gdn.plan(2, 37, 2, 64, 64) == (TC, 2)
+    assert gdn.plan(1, 75, 2, 64, 64) == (TC, 1)
+
+
+def test_plan_rules_that_hold_on_any_machine(monkeypatch):
+    monkeypatch.delenv("GDN_TC_CTAS", raising=False)
+    assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)          # a single frame: one CTA per head
+    assert gdn.plan(4, 16, 241, 1350, 128) == (SIMT, 1)    # D = 128: CUDA-core kernel
+    assert gdn.plan(1, 2, 8, 64, 32) == (SIMT, 1)          # D = 32
+    for forced in ("1", "2", "4"):
+        monkeypatch.setenv("GDN_TC_CTAS", forced)
+        assert gdn.plan(1, 32, 961, 880, 64) == (TC, int(forced))
+    monkeypatch.setenv("GDN_TC_CTAS", "3")                 # not a cluster size it builds
+    assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)
+    with pytest.raises(gdn.GdnError):
+        gdn.plan(1, 32, 961, 880, 48)
+
+
+def test_impl_override_routes_to_cuda_cores():
+    env = dict(os.environ, GDN_IMPL="simt")
+    env.pop("GDN_TC_CTAS", None)
+    code = ("from frame_wise_gated_scan_b200 import gdn; "
+            "print(gdn.plan(1, 32, 961, 880, 64))")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                         text=True, check=True).stdout.strip()
+    assert out == f"({SIMT}, 1)"
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(gdn, "_lib", None)
+    monkeypatch.setattr(gdn, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libgdn.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        gdn.lib()
+    with pytest.raises(RuntimeError, match="not built"):
+        gdn.plan(1, 32, 961, 880, 64)
