@@ -267,7 +267,7 @@ def main():
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", init_method="env://",
-                                timeout=__import__("datetime").timedelta(seconds=600))
+                                timeout=__import__("datetime").timedelta(seconds=300))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
 
