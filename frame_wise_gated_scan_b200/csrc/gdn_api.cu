@@ -45,6 +45,11 @@ int check_sizes(int B, int H, int T, int S, int D) {
 
 int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
   const int f = forced_kernel();
+  const int step = (f == GDN_KERNEL_SIMT) ? 0 : gdn::step_ctas_per_head(B, H, T, S, D);
+  if (step > 0) {
+    *ctas = step;
+    return GDN_KERNEL_STEP;
+  }
   const int tc = (f == GDN_KERNEL_SIMT) ? 0 : gdn::tc_ctas_per_head(B, H, T, S, D);
   if (tc > 0) {
     *ctas = tc;
@@ -60,7 +65,6 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
   if (flags & ~GDN_FLAG_NO_DELTA) return GDN_ERR_FLAGS;
-  if (noalloc && (long long)B * H > GDN_NOALLOC_MAX_HEADS) return GDN_ERR_SCRATCH;
   if (!q || !k || !v || !gamma || !beta || !out) return GDN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(gamma, 4) ||
@@ -73,6 +77,12 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
     return GDN_ERR_ALIAS;
   if (state_in && state_out && state_in != state_out && overlap(state_in, ns, state_out, ns))
     return GDN_ERR_ALIAS;
+  int ctas = 1;
+  const int kern = elt_bytes == 4 ? GDN_KERNEL_SIMT : choose_kernel(B, H, T, S, D, &ctas);
+  // The fixed scratch of the no-alloc call holds the transition-operand ring,
+  // which only the tensor-core kernel with more than one CTA per head uses.
+  if (noalloc && kern == GDN_KERNEL_TC && ctas > 1 && (long long)B * H > GDN_NOALLOC_MAX_HEADS)
+    return GDN_ERR_SCRATCH;
 
   gdn::Problem p;
   p.q = q;
@@ -96,9 +106,9 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   if (elt_bytes == 4) {
     err = gdn::launch_simt_f32(p);
   } else {
-    int ctas = 1;
-    const int kern = choose_kernel(B, H, T, S, D, &ctas);
-    if (kern != GDN_KERNEL_TC)
+    if (kern == GDN_KERNEL_STEP)
+      err = gdn::launch_step_bf16(p, ctas);   // allocates nothing
+    else if (kern != GDN_KERNEL_TC)
       err = gdn::launch_simt_bf16(p);   // allocates nothing either way
     else
       err = noalloc ? gdn::launch_tc_bf16_noalloc(p, ctas) : gdn::launch_tc_bf16(p, ctas);
@@ -164,6 +174,39 @@ int gdn_frame_step_f32_ex(const float* q, const float* k, const float* v, const 
   return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 4, false, flags);
 }
 
+int gdn_temporal_conv(const void* x, const float* w, const float* bias, const void* cache_in,
+                      void* cache_out, void* y, int B, int T, int S, int C, int frames_per_block,
+                      void* stream) {
+  if (B < 1 || T < 1 || S < 1 || C < 1 || frames_per_block < 1 || C % 8 != 0) return GDN_ERR_SHAPE;
+  const double elems = (double)B * T * S * C;
+  if (elems > 9.0e18 / 4.0) return GDN_ERR_SHAPE;
+  if (!x || !w || !y) return GDN_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(cache_in, 16) || !aligned(cache_out, 16) ||
+      !aligned(w, 4) || !aligned(bias, 4))
+    return GDN_ERR_ALIGN;
+  const size_t n = (size_t)B * T * S * C * 2;
+  const size_t nc = (size_t)B * S * C * 2;
+  if (overlap(y, n, x, n) || overlap(y, n, cache_in, nc) || overlap(y, n, cache_out, nc) ||
+      overlap(cache_out, nc, x, n))
+    return GDN_ERR_ALIAS;
+  if (cache_in && cache_out && cache_in != cache_out && overlap(cache_in, nc, cache_out, nc))
+    return GDN_ERR_ALIAS;
+  gdn::ConvProblem p;
+  p.x = x;
+  p.w = w;
+  p.bias = bias;
+  p.cache_in = cache_in;
+  p.cache_out = cache_out;
+  p.y = y;
+  p.B = B;
+  p.T = T;
+  p.S = S;
+  p.C = C;
+  p.F = frames_per_block;
+  p.stream = static_cast<cudaStream_t>(stream);
+  return gdn::launch_tconv_bf16(p) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head) {
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
@@ -175,7 +218,7 @@ int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head)
 int gdn_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
   unsigned int st = 0;
-  if (gdn::tc_read_status(&st) != cudaSuccess) return GDN_ERR_CUDA;
+  if (gdn::read_status(&st) != cudaSuccess) return GDN_ERR_CUDA;
   return st ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 

@@ -1,6 +1,7 @@
 // Internal interface between the C-ABI layer (gdn_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,7 +36,38 @@ cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head);
 // stream-ordered allocations (gdn_frame_scan_noalloc). Needs B * H <=
 // GDN_NOALLOC_MAX_HEADS; calls that overlap on the GPU race on the array.
 cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head);
-// Reads and clears the device status word of the tensor-core kernel.
-cudaError_t tc_read_status(unsigned int* status);
+
+// Row-split single-frame kernel (gdn_step.cu): T = 1, D = 64, a cluster of
+// CTAs per head sharing the frame's rows. Returns the CTAs per head for these
+// sizes, or 0 if it does not take them.
+int step_ctas_per_head(int B, int H, int T, int S, int D);
+cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head);
+
+// Causal temporal convolution (gdn_conv.cu), arrays as documented in include/gdn.h.
+struct ConvProblem {
+  const void* x;          // [B][T][S][C] bf16
+  const float* w;         // [C][3]
+  const float* bias;      // [C] or null
+  const void* cache_in;   // [B][S][C] bf16 or null
+  void* cache_out;        // [B][S][C] bf16 or null
+  void* y;                // [B][T][S][C] bf16
+  int B, T, S, C, F;
+  cudaStream_t stream;
+};
+cudaError_t launch_tconv_bf16(const ConvProblem& p);
+
+// Host helpers (gdn_host.cu).
+// TMA map of a [frames][S][D] bf16 array as the 3-D tensor (D, S, frames),
+// with 64-column (128-byte) x box_rows x 1 boxes and the 128-byte swizzle.
+// Rows past S inside a frame read as zero and are not stored.
+bool make_frame_map(CUtensorMap* m, const void* base, int D, int S, long long frames,
+                    int box_rows);
+// Device address of the status word on the current device (null on failure).
+unsigned int* status_word();
+// Reads and clears the device status word.
+cudaError_t read_status(unsigned int* status);
+// Bound of every device-side wait, in nanoseconds: 1 s. A build with
+// GDN_DEBUG reads GDN_DEBUG_WAIT_NS instead, so tests can make waits run out.
+unsigned long long wait_budget_ns();
 
 }  // namespace gdn

@@ -1,0 +1,505 @@
+// Row-split single-frame kernel of the frame-wise Gated DeltaNet update, bf16
+// inputs, D = 64: one frame per head (T = 1). This is the call of chunk-causal
+// rollout, where frames arrive one at a time and each one's latency counts
+// ("NVIDIA Apresenta SANA-WM ...", acheiumaia.com.br: the chunk-causal
+// autoregressive generator for sequential rollout, and the GDN item of
+// section "A Arquitetura").
+//
+// The update, with s = 1/sqrt(D*S), in the form the scan kernel also uses:
+//     M' = gamma M + A' M + c,  A' = -gamma beta s^2 K^T K,  c = beta s K^T V,
+//     O  = Q M'.
+// A frame is only S x D per tensor, so one CTA per head leaves most SMs idle
+// and streams its 450 KB alone. Here a thread-block cluster of P CTAs (P = 2
+// or 4) shares each head, and CTA r owns rows [r*chunk, (r+1)*chunk):
+//  1. one TMA burst loads its rows of K, V and Q (32-row boxes, 128-byte
+//     swizzle) while the threads copy the fp32 state M into shared memory;
+//  2. tcgen05: the partial K^T [K V] over its rows (M = 64, N = 128) into TMEM;
+//  3. reduce-scatter over distributed shared memory: CTA q receives every
+//     CTA's partial of state rows [q*64/P, (q+1)*64/P), by bulk copies that
+//     complete on q's mbarrier;
+//  4. CTA q sums them in a fixed order and updates its state rows on CUDA
+//     cores with the scan kernel's precision: A' and M rounded to bf16 for
+//     the product A' M, fp32 accumulation, gamma M and c added in fp32. It
+//     writes those rows of the final state;
+//  5. all-gather of M' in bf16 into every CTA of the cluster (bulk copies);
+//  6. tcgen05: O = Q M' for its own rows, TMEM -> bf16 -> TMA stores.
+//
+// Every wait is bounded. A wait that runs out records the role in the device
+// status word and raises an abort flag in every CTA of the cluster; the
+// remaining phases are skipped, every CTA drains the copies still in flight
+// towards it, and the kernel returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <atomic>
+
+#include "gdn.h"
+#include "gdn_internal.h"
+#include "gdn_wait.cuh"
+#include "sm100_ptx.h"
+
+namespace gdn {
+namespace {
+
+using namespace ptx;
+using namespace wait;
+
+constexpr int kD = 64;
+constexpr int kThreads = 256;
+constexpr int kBox = 32;                          // rows per TMA box (loads and stores)
+constexpr uint32_t kBoxBytes = kBox * kD * 2;     // 4 KB
+constexpr int kRowsMax = 384;                     // rows of a frame per CTA
+constexpr uint32_t kRegion = kRowsMax * kD * 2;   // 48 KB: one CTA's rows of K, V or Q
+constexpr uint32_t kTmemCols = 256;
+
+// Shared memory (from a 1 KB aligned base).
+constexpr uint32_t kOffK = 0;
+constexpr uint32_t kOffV = kRegion;
+constexpr uint32_t kOffQ = 2 * kRegion;
+constexpr uint32_t kOffM0 = 3 * kRegion;          // M (fp32, 64 x 64), 16 KB
+constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (64/P rows) x 512 B
+constexpr uint32_t kOffMg = kOffRed + 32768;      // M' in bf16: 64 rows x 128 B, 128-byte swizzle
+constexpr uint32_t kOffBar = kOffMg + 8192;
+enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarGather, kBarO, kBarDrain, kNumBars };
+constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
+constexpr uint32_t kBytes = kOffAbort + 16;
+constexpr uint32_t kSmemAlloc = kBytes + 1024;    // base alignment slack
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0, "swizzled regions are 1 KB aligned");
+
+// Regions reused once the partial product has read K (K region) and V (V region):
+constexpr uint32_t kOffM0r = kOffK;               // M rounded to bf16, as fp32, 16 KB
+constexpr uint32_t kOffArow = kOffK + 16384;      // A' rows (fp32 holding bf16 values), <= 8 KB
+constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
+constexpr uint32_t kOffMst = kOffK + 32768;       // own rows of M' in bf16, <= 4 KB
+constexpr uint32_t kOffSend = kOffV;              // partial product, 64 rows x 512 B
+constexpr uint32_t kOffOut = kOffV;               // output tiles, 3 x 16 KB (after the gather)
+
+// Status bits (shared with the scan kernel's numbering scheme, high bits).
+enum : uint32_t {
+  kStLoad = 1u << 16, kStMma = 1u << 17, kStRed = 1u << 18, kStGather = 1u << 19,
+  kStOut = 1u << 20, kStDrain = 1u << 21, kStConfig = 1u << 22
+};
+
+struct StepParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_o;
+  const float* gamma;
+  const float* beta;
+  const float* state_in;
+  float* state_out;
+  unsigned int* status;
+  unsigned long long timeout_ns;   // bound of every wait
+  int S;
+  int chunk;      // rows per CTA (multiple of 32); CTA r owns [r*chunk, min(S, (r+1)*chunk))
+  float s;        // key scale 1/sqrt(D*S)
+  float s2;       // its square
+  float delta;    // 1: delta rule; 0: GDN_FLAG_NO_DELTA (A' = 0)
+};
+
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in 128-byte rows with the
+// 128-byte swizzle (the layout TMA writes and the tcgen05 descriptors read).
+__device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t chunk) {
+  const uint32_t off = row * 128u + chunk * 16u;
+  return off ^ (((off >> 7) & 7u) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_constant__ StepParams p) {
+  constexpr int R = kD / P;   // state rows this CTA updates
+  static_assert(R % 16 == 0, "a warp's 16 rows go to one CTA");
+  extern __shared__ uint8_t smem_raw[];
+  {
+    // Wrong launch shape: record it and touch nothing (uniform over the cluster).
+    uint32_t dsmem;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dsmem));
+    if (blockDim.x != kThreads || blockDim.y != 1 || blockDim.z != 1 || dsmem < kSmemAlloc ||
+        cluster_nctarank() != (uint32_t)P) {
+      if (threadIdx.x == 0) atomicOr(p.status, kStConfig);
+      return;
+    }
+  }
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int bh = blockIdx.x / P;
+  const int r0 = (int)rank * p.chunk;
+  const int r1 = min(p.S, r0 + p.chunk);
+  const int nrows = max(0, r1 - r0);
+  const int nbox = (nrows + kBox - 1) / kBox;
+  const int nq = (nrows + 127) / 128;   // 128-row read-out tiles
+  auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * i; };
+  Ctl ctl{sb + kOffAbort, p.status, p.timeout_ns, P};
+  const float g = __ldg(p.gamma + bh);
+  const float be = __ldg(p.beta + bh);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
+    fence_mbar_init();
+    // The exchange barriers are armed before the cluster barrier below, and
+    // peers only send after it.
+    mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
+    mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
+    if (nbox > 0) {
+      const uint64_t pol = policy_evict_first();   // read once
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
+      for (int b = 0; b < nbox; ++b) {
+        tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, bh, pol);
+        tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, bh, pol);
+      }
+      mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
+      for (int b = 0; b < nbox; ++b)
+        tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, bh, pol);
+    }
+  }
+  // The initial state, whole, in every CTA. It is read here, before the first
+  // cluster barrier, and the final state is written only after it: so
+  // state_in == state_out is safe.
+  {
+    const float4* src = reinterpret_cast<const float4*>(p.state_in + (size_t)bh * kD * kD);
+    for (int i = threadIdx.x; i < kD * kD / 4; i += kThreads) {
+      const float4 x = p.state_in ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kOffM0 + 16u * i),
+                   "f"(x.x), "f"(x.y), "f"(x.z), "f"(x.w)
+                   : "memory");
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + kOffTmemPtr, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();   // every CTA's barriers are initialised and armed
+  const uint32_t tmem = ld_shared_u32(sb + kOffTmemPtr);
+  bool issued_mma = false;
+
+  // ---------------------------------------------------------------- 2. partial K^T [K V]
+  if (warp == 1 && lane == 0 && nbox > 0) {
+    if (wait_bar(bar(kBarKv), 0, ctl, kStLoad)) {
+      tc_fence_after();
+      // A = K^T (M = 64 key dims, one 128-byte atom), B = [K V] (N = 128: the K
+      // and V regions are its two atoms, kRegion apart); both MN-major views of
+      // the row-major tiles; 16 rows per MMA.
+      constexpr uint32_t idesc = idesc_bf16(64, 128, 1, 1);
+      for (int kk = 0; kk < 2 * nbox; ++kk) {
+        const uint64_t a = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
+        const uint64_t b = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
+        mma_bf16(tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar(kBarMma));
+      issued_mma = true;
+    }
+  }
+
+  // ---------------------------------------------------------------- 3. reduce-scatter
+  // With M = 64 the accumulator row i (key dim) sits in TMEM lane 32(i/16) + i%16:
+  // warp w (< 4) reads lanes 32w.., and its lanes 0-15 hold key rows 16w..16w+15,
+  // columns 0-63 = K^T K, 64-127 = K^T V. Those 16 rows (8 KB of fp32) go to the
+  // CTA that updates them, staged with chunk c of row i at chunk c ^ (i & 7).
+  if (warp < 4) {
+    const bool ok = nbox == 0 || warp_wait(bar(kBarMma), 0, ctl, kStMma);
+    if (ok) {
+      tc_fence_after();
+      const int il = lane & 15;
+      const uint32_t row_addr = sb + kOffSend + (uint32_t)(warp * 16 + il) * 512u;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[64];
+        if (nbox > 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tmem + 64 * h + 16 * c + ((uint32_t)(warp * 32) << 16), r16);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+          }
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) v[e] = 0u;
+        }
+        if (lane < 16) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t cc = 16 * h + c;
+            st_shared_v4(row_addr + ((cc ^ (uint32_t)(il & 7)) << 4),
+                         make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_cta();   // staged rows visible to the bulk copy
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t dst = (uint32_t)(warp * P / 4);
+        const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
+        bulk_copy_to_cluster(mapa(sb + kOffRed + slot_row * 512u, dst),
+                             sb + kOffSend + (uint32_t)warp * 16u * 512u, 16u * 512u,
+                             mapa(bar(kBarRed), dst));
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- 4. recurrence, own rows
+  const bool red_ok = warp_wait(bar(kBarRed), 0, ctl, kStRed);
+  __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
+  if (red_ok && !aborted(ctl)) {
+    const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 K^T K (0 without delta)
+    const float cbs = be * p.s;                    // c = beta s K^T V
+    for (int e = threadIdx.x; e < R * 128; e += kThreads) {
+      const int il = e >> 7, n = e & 127;
+      const uint32_t off = (uint32_t)((((n >> 2) ^ (il & 7)) << 4) + (n & 3) * 4);
+      float sum = 0.f;
+#pragma unroll
+      for (int src = 0; src < P; ++src)
+        sum += ld_shared_f32(sb + kOffRed + (uint32_t)(src * R + il) * 512u + off);
+      if (n < kD)
+        st_shared_f32(sb + kOffArow + (uint32_t)(il * kD + n) * 4u, bf16_round(coef * sum));
+      else
+        st_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + n - kD) * 4u, cbs * sum);
+    }
+    for (int e = threadIdx.x; e < kD * kD; e += kThreads)
+      st_shared_f32(sb + kOffM0r + 4u * e, bf16_round(ld_shared_f32(sb + kOffM0 + 4u * e)));
+  }
+  __syncthreads();
+  if (red_ok && !aborted(ctl)) {
+    const int j = threadIdx.x & 63;      // value column
+    const int ib = threadIdx.x >> 6;     // rows ib, ib + 4, ...
+    constexpr int NR = R / 4;
+    float acc[NR];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) acc[n] = 0.f;
+    if (p.delta != 0.f) {
+#pragma unroll 8
+      for (int k = 0; k < kD; ++k) {
+        const float mk = ld_shared_f32(sb + kOffM0r + (uint32_t)(k * kD + j) * 4u);
+#pragma unroll
+        for (int n = 0; n < NR; ++n)
+          acc[n] = fmaf(ld_shared_f32(sb + kOffArow + (uint32_t)((ib + 4 * n) * kD + k) * 4u), mk, acc[n]);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      const int il = ib + 4 * n;
+      const int gi = (int)rank * R + il;
+      const float m0 = ld_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u);
+      const float m1 = fmaf(g, m0, acc[n]) + ld_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + j) * 4u);
+      if (p.state_out) p.state_out[((size_t)bh * kD + gi) * kD + j] = m1;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(m1);
+      st_shared_u16(sb + kOffMst + swz128((uint32_t)il, (uint32_t)(j >> 3)) + (uint32_t)(j & 7) * 2u,
+                    *reinterpret_cast<const uint16_t*>(&hb));
+    }
+  }
+  fence_proxy_async_cta();   // M' rows visible to the bulk copies
+  __syncthreads();
+  // ---------------------------------------------------------------- 5. all-gather of M' (bf16)
+  if (threadIdx.x == 0 && red_ok && !aborted(ctl)) {
+    for (int d = 0; d < P; ++d)
+      bulk_copy_to_cluster(mapa(sb + kOffMg + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
+                           (uint32_t)R * 128u, mapa(bar(kBarGather), (uint32_t)d));
+  }
+
+  // ---------------------------------------------------------------- 6. read-out O = Q M'
+  if (warp == 1 && lane == 0 && nq > 0) {
+    if (wait_bar(bar(kBarGather), 0, ctl, kStGather) && wait_bar(bar(kBarQ), 0, ctl, kStLoad)) {
+      tc_fence_after();
+      constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);   // Q K-major, M' MN-major
+      for (int i = 0; i < nq; ++i) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = smem_desc(sb + kOffQ + i * 16384 + kk * 32, 16, 1024, 2);
+          const uint64_t b = smem_desc(sb + kOffMg + kk * 2048, 8192, 1024, 2);
+          mma_bf16(tmem + 64 * i, a, b, id_o, kk > 0 ? 1u : 0u);
+        }
+      }
+      mma_commit(bar(kBarO));
+      issued_mma = true;
+    }
+  }
+  // Output tiles: warps 4g..4g+3 take tiles g, g + 2, ...; lane l of warp
+  // quarter q holds tile row 32q + l.
+  {
+    const int grp = warp >> 2;
+    const int qd = warp & 3;
+    if (grp < nq) {
+      const bool ok = warp_wait(bar(kBarO), 0, ctl, kStOut);
+      if (ok) {
+        tc_fence_after();
+        for (int i = grp; i < nq; i += 2) {
+          uint32_t v[64];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tmem + 64 * i + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+          }
+          tmem_wait_ld();
+          const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+          const uint32_t row = (uint32_t)(qd * 32 + lane);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+            st_shared_v4(tile + swz128(row, (uint32_t)c), w);
+          }
+        }
+        tc_fence_before();
+        fence_proxy_async_cta();
+      }
+      named_bar_sync(1 + grp, 128);   // every warp of the group arrives, ok or not
+      if (qd == 0 && lane == 0 && !aborted(ctl)) {
+        const uint64_t pol = policy_evict_first();
+        for (int i = grp; i < nq; i += 2) {
+          const int y0 = r0 + 128 * i;
+          const int y1 = min(r1, y0 + 128);
+          const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+          for (int y = y0; y < y1; y += kBox)
+            tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, bh, pol);
+        }
+        bulk_commit();
+        bulk_wait0();
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- exit
+  if (warp == 1 && lane == 0 && issued_mma) {   // every MMA done before TMEM is freed
+    mma_commit(bar(kBarDrain));
+    drain_bar(bar(kBarDrain), 0, ctl, kStDrain);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // normal path: every copy into each CTA has landed (each waited for it)
+  if (aborted(ctl)) {
+    // Same verdict in every CTA (the flag is raised in all of them before the
+    // raising thread reaches the barrier above). Let copies still in flight
+    // land before any CTA of the cluster leaves: loads issued here, and bulk
+    // copies from peers (all issued before that barrier).
+    if (threadIdx.x == 0) {
+      if (nbox > 0) {
+        drain_bar(bar(kBarKv), 0, ctl, kStDrain);
+        drain_bar(bar(kBarQ), 0, ctl, kStDrain);
+      }
+      drain_bar(bar(kBarRed), 0, ctl, kStDrain);
+      drain_bar(bar(kBarGather), 0, ctl, kStDrain);
+    }
+    __syncthreads();
+    cluster_sync();
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int P>
+cudaError_t prepare() {
+  static std::atomic<bool> done[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gdn_step_kernel<P>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+int chunk_rows(int S, int P) {
+  const int per = (S + P - 1) / P;
+  return (per + kBox - 1) / kBox * kBox;
+}
+
+template <int P>
+cudaError_t launch_p(const Problem& pr) {
+  cudaError_t e = prepare<P>();
+  if (e != cudaSuccess) return e;
+  StepParams p;
+  const long long frames = (long long)pr.B * pr.H;
+  if (!make_frame_map(&p.tm_q, pr.q, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p.tm_k, pr.k, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p.tm_v, pr.v, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p.tm_o, pr.out, kD, pr.S, frames, kBox))
+    return cudaErrorInvalidValue;
+  p.status = status_word();
+  if (!p.status) return cudaErrorInvalidDevice;
+  p.gamma = pr.gamma;
+  p.beta = pr.beta;
+  p.state_in = pr.state_in;
+  p.state_out = pr.state_out;
+  p.timeout_ns = wait_budget_ns();
+  p.S = pr.S;
+  p.chunk = chunk_rows(pr.S, P);
+  p.s = pr.key_scale;
+  p.s2 = (float)(1.0 / ((double)kD * (double)pr.S));
+  p.delta = pr.delta ? 1.f : 0.f;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(frames * P), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = pr.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gdn_step_kernel<P>, p);
+}
+
+}  // namespace
+
+int step_ctas_per_head(int B, int H, int T, int S, int D) {
+  if (D != kD || T != 1) return 0;
+  const long long heads = (long long)B * H;
+  if (heads * 4 > (1ll << 31) - 1) return 0;
+  int P = 4;
+  // Tuning override: GDN_STEP_CTAS=2|4 forces the cluster size; 0 turns this
+  // kernel off (single frames then run on the scan kernels).
+  if (const char* e = getenv("GDN_STEP_CTAS")) {
+    const int v = atoi(e);
+    if (e[0] == '0' && v == 0) return 0;
+    if (v == 2 || v == 4) P = v;
+  }
+  if (chunk_rows(S, P) > kRowsMax) P = 4;
+  if (chunk_rows(S, P) > kRowsMax) return 0;
+  return P;
+}
+
+cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head) {
+  if (p.T != 1 || p.D != kD) return cudaErrorInvalidValue;
+  switch (ctas_per_head) {
+    case 2: return launch_p<2>(p);
+    case 4: return launch_p<4>(p);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gdn

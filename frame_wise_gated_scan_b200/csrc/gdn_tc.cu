@@ -52,8 +52,6 @@
 
 namespace gdn {
 
-__device__ unsigned int g_tc_status = 0;
-
 #ifdef GDN_TRACE
 // Event timeline of head 0's cluster (globaltimer ns), for pipeline analysis
 // builds only: [rank][event][frame or own-frame index].
@@ -99,7 +97,7 @@ constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 constexpr int kRing = 16;                                       // frames per head in the ring
 constexpr int kStoreRows = 16;                                  // rows per output store box
 
-// Status codes recorded in g_tc_status (bit per waiting role).
+// Status codes recorded in the device status word (bit per waiting role).
 enum : uint32_t {
   kStKvLoad = 1u << 0, kStQLoad = 1u << 1, kStMma = 1u << 2, kStChain = 1u << 3,
   kStProd = 1u << 4, kStOut = 1u << 5, kStDrain = 1u << 6, kStMoEmpty = 1u << 7,
@@ -429,6 +427,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     tmem_alloc(tmem_ptr, L::TMEM_COLS);
     tmem_relinquish();
   }
+  // The recurrence warps read the initial state before the cluster barrier
+  // below. Rank 0 writes the final state only after that barrier, so with
+  // state_in == state_out no CTA of the head can read a row rank 0 has
+  // already overwritten. Lane l of warp quarter q owns row 16q + (l % 16),
+  // value columns 32 (l / 16) .. + 32.
+  float m[32];
+  if (warp >= 4 && warp < 8) {
+    const int row = (warp & 3) * 16 + (lane & 15);
+    const int col0 = 32 * (lane >> 4);
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj)
+      m[jj] = p.state_in ? p.state_in[((size_t)bh * kD + row) * kD + col0 + jj] : 0.f;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -669,10 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int qd = warp & 3;
     const int hf = lane >> 4;
     const int row = qd * 16 + (lane & 15);
-    float m[32];                               // fp32 state, row `row`, columns 32hf..32hf+31
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj)
-      m[jj] = p.state_in ? p.state_in[((size_t)bh * kD + row) * kD + 32 * hf + jj] : 0.f;
+    // m: the fp32 state, row `row`, columns 32hf..32hf+31 (loaded before the
+    // first cluster barrier)
     auto store_state = [&](uint32_t buf) {
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -947,38 +956,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver's tensor-map encoder, looked up once per process.
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// [B*H*T][S][64] bf16 viewed as a 3-D tensor (64, S, B*H*T); 64 x 128 x 1 boxes with
-// the 128-byte swizzle. Rows past S inside a frame read as zero and are not stored.
+// [B*H*T][S][64] bf16 viewed as a 3-D tensor (64, S, B*H*T); 64 x box_rows x 1
+// boxes with the 128-byte swizzle. Rows past S inside a frame read as zero and
+// are not stored.
 bool make_map(CUtensorMap* m, const void* base, int S, long long frames, int box_rows = kTile) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S, (cuuint64_t)frames};
-  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S * kD * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)box_rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_frame_map(m, base, kD, S, frames, box_rows);
 }
 
 template <int P>
@@ -1033,21 +1015,6 @@ int resident_clusters() {
   cudaGetLastError();
   cache[dev].store(n + 2, std::memory_order_release);
   return n;
-}
-
-// Address of the device status word on the current device, looked up once per device.
-unsigned int* status_word() {
-  static std::atomic<unsigned int*> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  unsigned int* a = cache[dev].load(std::memory_order_acquire);
-  if (!a) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_tc_status) != cudaSuccess) return nullptr;
-    a = static_cast<unsigned int*>(ptr);
-    cache[dev].store(a, std::memory_order_release);
-  }
-  return a;
 }
 
 // Address of g_noalloc_scratch on the current device. cudaGetSymbolAddress
@@ -1210,12 +1177,5 @@ extern "C" __attribute__((visibility("default"))) int gdn_trace_heads_copy(void*
   return cudaMemcpyFromSymbol(dst, g_trace_heads, n) == cudaSuccess ? (int)n : -1;
 }
 #endif
-
-cudaError_t tc_read_status(unsigned int* status) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(status, g_tc_status, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(unsigned int));
-}
 
 }  // namespace gdn

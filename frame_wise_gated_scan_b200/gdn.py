@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
 
 KERNEL_SIMT = 1
 KERNEL_TC = 2
+KERNEL_STEP = 3
 FLAG_NO_DELTA = 1     # GDN_FLAG_NO_DELTA: R = V, the decayed cumulative (block KV cache) form
 
 _lib = None
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = i
+        L.gdn_temporal_conv.argtypes = [vp, fp, fp, vp, vp, vp, i, i, i, i, i, vp]
+        L.gdn_temporal_conv.restype = i
         L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
         L.gdn_plan.restype = i
         L.gdn_device_status.argtypes = []
@@ -206,6 +209,45 @@ def frame_step(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
     delta=False as in frame_scan."""
     return _call(True, q, k, v, gamma, beta, state_in, out, state_out, want_state,
                  flags=0 if delta else FLAG_NO_DELTA)
+
+
+def temporal_conv(x, w, bias=None, cache_in=None, *, frames_per_block=None, y=None,
+                  cache_out=None, want_cache=True):
+    """Causal temporal convolution with a carried last-frame cache
+    (gdn_temporal_conv). x: [B,T,S,C] bf16 CUDA tensor; w: [C,3] fp32 taps for
+    the previous, current and next frame; bias: [C] fp32 or None; cache_in:
+    [B,S,C] bf16 (the previous call's last frame) or None for zeros;
+    frames_per_block: block length (None: the whole call is one block).
+    cache_out may be cache_in. Returns (y, cache_out); cache_out is None if
+    want_cache is False and none was given."""
+    if x.dim() != 4 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a [B,T,S,C] bfloat16 tensor")
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("x must be a CUDA tensor")
+    B, T, S, C = x.shape
+    _check(x, "x", torch.bfloat16, (B, T, S, C), device)
+    _check(w, "w", torch.float32, (C, 3), device)
+    if bias is not None:
+        _check(bias, "bias", torch.float32, (C,), device)
+    if cache_in is not None:
+        _check(cache_in, "cache_in", torch.bfloat16, (B, S, C), device)
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _check(y, "y", torch.bfloat16, (B, T, S, C), device)
+    if cache_out is None and want_cache:
+        cache_out = torch.empty((B, S, C), dtype=torch.bfloat16, device=device)
+    elif cache_out is not None:
+        _check(cache_out, "cache_out", torch.bfloat16, (B, S, C), device)
+    F = T if frames_per_block is None else int(frames_per_block)
+    L = lib()
+    with torch.cuda.device(device):
+        st = L.gdn_temporal_conv(_ptr(x), _ptr(w), _ptr(bias), _ptr(cache_in), _ptr(cache_out),
+                                 _ptr(y), B, T, S, C, F, _stream_handle(device))
+    if st != 0:
+        raise GdnError(st, "gdn_temporal_conv")
+    return y, cache_out
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,

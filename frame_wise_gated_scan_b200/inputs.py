@@ -195,3 +195,67 @@ def flops(wl: Workload, T: int | None = None) -> int:
     """Floating-point operations of the three S-by-D-by-D contractions per frame and head."""
     T = wl.T if T is None else T
     return 6 * wl.heads * T * wl.S * wl.D * wl.D
+
+
+# ---- the causal temporal convolution (the companion of the GDN state in
+# chunk-causal rollout): x [B][T][S][C] bf16, taps w [C][3] and bias [C] fp32,
+# a carried last-frame cache [B][S][C] bf16.
+
+@dataclasses.dataclass(frozen=True)
+class ConvWorkload:
+    name: str
+    B: int
+    T: int
+    S: int
+    C: int
+    F: int        # frames per block
+    seed: int
+
+    def with_(self, **kw) -> "ConvWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+# The rollout's shapes: 961 latent frames of 22 x 40 tokens, C = 2048 channels
+# (32 heads x 64, the width of the GDN layer), blocks of 8 frames.
+CONV_WORKLOADS = {
+    "conv_rollout": ConvWorkload("conv_rollout", 1, 961, 880, 2048, 8, 7),
+}
+
+
+def conv_frame(wl: ConvWorkload, b: int, t: int) -> np.ndarray:
+    """Frame t of sequence b: float32 [S, C] holding bf16 values, N(0, 1)."""
+    rng = _rng(wl.seed, b, t, 0)
+    return bf16_to_f32(bf16_round(rng.standard_normal((wl.S, wl.C), dtype=np.float32)))
+
+
+def conv_params(wl: ConvWorkload):
+    """Taps w [C, 3] ~ N(0, 1/3) and bias [C] ~ N(0, 0.01), float32."""
+    rng = _rng(wl.seed + 2000, 0, 0, 0)
+    w = (rng.standard_normal((wl.C, 3), dtype=np.float32) / np.float32(math.sqrt(3.0)))
+    bias = rng.standard_normal((wl.C,), dtype=np.float32) * np.float32(0.1)
+    return w.astype(np.float32), bias.astype(np.float32)
+
+
+def conv_cache(wl: ConvWorkload) -> np.ndarray:
+    """A carried cache [B, S, C]: float32 holding bf16 values, N(0, 1)."""
+    out = np.empty((wl.B, wl.S, wl.C), np.float32)
+    for b in range(wl.B):
+        rng = _rng(wl.seed + 1000, b, 0, 0)
+        out[b] = bf16_to_f32(bf16_round(rng.standard_normal((wl.S, wl.C), dtype=np.float32)))
+    return out
+
+
+def conv_full(wl: ConvWorkload) -> np.ndarray:
+    """Whole input x [B, T, S, C] float32 (small workloads)."""
+    x = np.empty((wl.B, wl.T, wl.S, wl.C), np.float32)
+    for b in range(wl.B):
+        for t in range(wl.T):
+            x[b, t] = conv_frame(wl, b, t)
+    return x
+
+
+def conv_bytes(wl: ConvWorkload) -> int:
+    """Bytes one call must move: x read and y written once (bf16), the taps
+    and bias, the cache read and written."""
+    n = wl.B * wl.T * wl.S * wl.C
+    return 2 * n * 2 + wl.C * 16 + 2 * wl.B * wl.S * wl.C * 2

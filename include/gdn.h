@@ -70,7 +70,7 @@ typedef enum gdn_status {
   GDN_ERR_CUDA = -5,            /* a CUDA runtime or driver call failed */
   GDN_ERR_TIMEOUT = -6,         /* a device-side wait ran out (from gdn_device_status) */
   GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
-  GDN_ERR_SCRATCH = -8,         /* B * H > GDN_NOALLOC_MAX_HEADS (gdn_frame_scan_noalloc) */
+  GDN_ERR_SCRATCH = -8,         /* gdn_frame_scan_noalloc: a ring plan with B * H > GDN_NOALLOC_MAX_HEADS */
   GDN_ERR_FLAGS = -9            /* unknown bits in `flags` (the _ex calls) */
 } gdn_status;
 
@@ -90,8 +90,14 @@ GDN_API int gdn_frame_scan(const void* q, const void* k, const void* v,
 
 /* One bf16 frame (T = 1) for chunk-causal rollout: the state is read from
  * state_in and written to state_out, which may be the same buffer, so a
- * caller can carry it across calls. Same arithmetic as gdn_frame_scan; a chain
- * of steps gives the same result as one scan over the same frames. */
+ * caller can carry it across calls. This is the sequential rollout variant
+ * the SANA-WM article names among its three inference modes ("NVIDIA
+ * Apresenta SANA-WM ...", acheiumaia.com.br, the paragraph on the
+ * bidirectional, chunk-causal autoregressive and distilled generators): one
+ * latent frame arrives per call and the constant-size D x D state carries the
+ * whole history. Same update and precision as gdn_frame_scan (the
+ * state-dependent product takes A' and M in bf16); a chain of steps matches
+ * one scan over the same frames to fp32 rounding. */
 GDN_API int gdn_frame_step(const void* q, const void* k, const void* v,
                    const float* gamma, const float* beta,
                    const float* state_in, float* state_out, void* out,
@@ -112,8 +118,12 @@ GDN_API int gdn_frame_step(const void* q, const void* k, const void* v,
  * fixed array in the library's device code instead, and calls no cudaMalloc,
  * cudaMallocAsync, cudaFree or cudaFreeAsync.
  *
- * Limit: B * H <= GDN_NOALLOC_MAX_HEADS (32); larger sizes return
- * GDN_ERR_SCRATCH and enqueue nothing. The array holds 16 frames x 24 KiB of
+ * Limit: the scratch is the transition-operand ring, which only a plan with
+ * the tensor-core kernel and more than one CTA per head uses (gdn_plan). For
+ * such a plan B * H must be <= GDN_NOALLOC_MAX_HEADS (32); a larger one
+ * returns GDN_ERR_SCRATCH, after the argument checks every entry point makes,
+ * and enqueues nothing. Other plans take no scratch and have no limit. The
+ * array holds 16 frames x 24 KiB of
  * transition operands plus 160 bytes of flags per head: 12 MiB + 5 KiB,
  * reserved on each device when the library's device code is loaded there,
  * whether or not this entry point is called. The first call on a device looks
@@ -176,12 +186,42 @@ GDN_API int gdn_frame_step_f32_ex(const float* q, const float* k, const float* v
                        const float* state_in, float* state_out, float* out,
                        int B, int H, int S, int D, unsigned int flags, void* stream);
 
+/* Causal temporal convolution with a carried last-frame cache, the companion
+ * of the GDN state in chunk-causal rollout ("SANA-Video" ICLR 2026 oral
+ * transcript, shadowingenglish.com, the part on the causal FFN with temporal
+ * convolution: a zero token is padded between two blocks so that a block
+ * cannot see the next one, and the last token of a block is cached as the
+ * first token the next block sees). Three depthwise taps along the frame
+ * axis, centred on the current frame. Per channel c, token s, frame t, with
+ * blocks of frames_per_block frames counted from the call's first frame:
+ *
+ *     y[t] = w[c][0] x_prev + w[c][1] x[t] + w[c][2] x_next + bias[c]
+ *
+ *   x_prev = x[t-1]; for t = 0, cache_in (the previous call's last frame;
+ *            NULL means zero, the start of a video)
+ *   x_next = x[t+1] inside a block; 0 for the last frame of a block (and of
+ *            the call)
+ *
+ * cache_out receives x[T-1] (NULL: not written), so consecutive calls over
+ * whole blocks equal one call. Layouts: x, y [B][T][S][C] bf16; w [C][3] and
+ * bias [C] (or NULL) fp32; cache_in, cache_out [B][S][C] bf16. Arithmetic in
+ * fp32, y rounded to bf16 (nearest even). C must be a multiple of 8
+ * (GDN_ERR_SHAPE); x, y and the caches 16-byte aligned, w and bias 4-byte
+ * aligned (GDN_ERR_ALIGN); y must not overlap x or the caches, cache_out must
+ * not overlap x, and cache_in may equal cache_out (GDN_ERR_ALIAS). Device
+ * pointers, stream-ordered like the other calls; allocates nothing. */
+GDN_API int gdn_temporal_conv(const void* x, const float* w, const float* bias,
+                              const void* cache_in, void* cache_out, void* y,
+                              int B, int T, int S, int C, int frames_per_block, void* stream);
+
 /* Which kernel a bf16 call with these sizes runs, without running it.
  * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head
  * (the thread-block cluster size, 1 for the CUDA-core kernel).
  * Returns GDN_OK or the error the call itself would return for the sizes. */
 #define GDN_KERNEL_SIMT 1   /* CUDA-core kernel, one CTA per 16 state columns */
 #define GDN_KERNEL_TC 2     /* tcgen05 kernel, a cluster of CTAs per head */
+#define GDN_KERNEL_STEP 3   /* single-frame tcgen05 kernel (T = 1, D = 64): a cluster of
+                               CTAs per head splits the frame's rows */
 GDN_API int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head);
 
 /* Synchronizes the current device, then returns GDN_ERR_TIMEOUT if any kernel

@@ -9,6 +9,7 @@ import torch
 
 from frame_wise_gated_scan_b200 import gdn, inputs
 from gpu_util import (TOL_BF16, TOL_F32, assert_close, device_workload, oracle_head, to_np64)
+from oracle import gdn_scan_ref, rel_frobenius
 
 pytestmark = pytest.mark.gpu
 
@@ -16,10 +17,11 @@ _cache = {}
 
 
 def workload_on_device(name, T=None):
-    key = (name, T)
+    wl = name if isinstance(name, inputs.Workload) else inputs.WORKLOADS[name]
+    key = (wl, T)
     if key not in _cache:
         _cache.clear()           # keep one large workload resident at a time
-        _cache[key] = device_workload(inputs.WORKLOADS[name], T)
+        _cache[key] = device_workload(wl, T)
     return _cache[key]
 
 
@@ -218,3 +220,94 @@ def test_no_delta_differs_from_delta_and_step_chain_equals_scan():
     assert gdn.device_status() == 0
     e = float((state - st_n).norm() / st_n.norm())
     assert e <= 1e-6, f"no-delta step chain vs scan: {e:.3e}"
+
+
+# ---- the tensor-core kernel on the inputs where its bf16 operands are weakest ----
+
+# The stress recipe (key norms unit * exp(N(0,1)), gamma ~ U(.99,1), beta = 1)
+# at D = 64, so that it runs on the tcgen05 kernel: near-unit decay gives the
+# longest memory, and large aligned keys the largest |A'| = gamma beta s^2 |K^T K|,
+# which is where rounding A' and M to bf16 in A' M could add up.
+STRESS_D64 = inputs.Workload("stress_d64", 2, 4, 64, 241, 1350, "bf16", 5, "lognormal", "stress")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("ctas", ["1", "2", "4"])
+def test_tensor_core_stress_recipe_d64(monkeypatch, ctas):
+    monkeypatch.setenv("GDN_TC_CTAS", ctas)
+    wl = STRESS_D64
+    assert gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D) == (gdn.KERNEL_TC, int(ctas))
+    q, k, v, g, be = workload_on_device(wl)
+    out, st = gdn.frame_scan(q, k, v, g, be)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert torch.isfinite(out).all() and torch.isfinite(st).all(), "stress d64: NaN/Inf"
+    worst_o = worst_s = 0.0
+    for b, h in [(0, 0), (0, 3), (1, 1), (1, 2)]:
+        ro, rs = oracle_head(wl, b, h)
+        eo, es = assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16,
+                              f"stress d64 P={ctas} b{b} h{h}")
+        worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
+    print(f"stress recipe D=64 P={ctas}: worst per-frame out error {worst_o:.3e}, "
+          f"final state {worst_s:.3e}")
+
+
+@pytest.mark.parametrize("ctas", ["1", "2", "4"])
+def test_tensor_core_gamma1_beta0_keeps_the_state(monkeypatch, ctas):
+    """gamma = 1, beta = 0: every update leaves M_0 unchanged (A' = 0, c = 0,
+    and 1 * m + 0 is exact in fp32), so the final state equals M_0 bit for bit
+    and every frame reads out Q_t M_0."""
+    monkeypatch.setenv("GDN_TC_CTAS", ctas)
+    wl = inputs.Workload("literal", 1, 4, 64, 40, 300, "bf16", 530, "lognormal", "stress")
+    assert gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D) == (gdn.KERNEL_TC, int(ctas))
+    q, k, v, _, _ = device_workload(wl)
+    g = torch.ones((wl.B, wl.H, wl.T), device="cuda")
+    be = torch.zeros_like(g)
+    m0 = inputs.state(wl)
+    out, st = gdn.frame_scan(q, k, v, g, be, torch.from_numpy(m0).cuda())
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert torch.equal(st.cpu(), torch.from_numpy(m0)), "state changed with beta = 0, gamma = 1"
+    for b, h in [(0, 0), (0, 3)]:
+        qh, kh, vh, _, _ = inputs.head(wl, b, h)
+        ro, rs = gdn_scan_ref(qh, kh, vh, np.ones(wl.T), np.zeros(wl.T), state_in=m0[b, h])
+        assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16, f"literal h{h}")
+
+
+@pytest.mark.parametrize("ctas", ["1", "2", "4"])
+def test_tensor_core_beta0_decays_by_gamma_products(monkeypatch, ctas):
+    """beta = 0: M_t = (gamma_1 ... gamma_t) M_0. In fp32 the state takes one
+    rounding per frame, so it stays within T * 2^-24 of the product."""
+    monkeypatch.setenv("GDN_TC_CTAS", ctas)
+    wl = inputs.Workload("decay", 1, 4, 64, 60, 200, "bf16", 531, "l2", "rollout")
+    q, k, v, g, _ = device_workload(wl)
+    be = torch.zeros_like(g)
+    m0 = inputs.state(wl)
+    out, st = gdn.frame_scan(q, k, v, g, be, torch.from_numpy(m0).cuda())
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    gam = g.double().cpu().numpy()
+    for b, h in [(0, 1), (0, 2)]:
+        expect = np.prod(gam[b, h]) * m0[b, h].astype(np.float64)
+        e = float(np.max(rel_frobenius(to_np64(st[b, h]), expect)))
+        assert e <= wl.T * 2.0 ** -23, f"beta = 0 decay h{h}: state error {e:.3e}"
+        qh, kh, vh, gh, _ = inputs.head(wl, b, h)
+        ro, rs = gdn_scan_ref(qh, kh, vh, gh, np.zeros(wl.T), state_in=m0[b, h])
+        assert_close(to_np64(out[b, h]), ro, None, None, TOL_BF16, f"decay h{h}")
+
+
+@pytest.mark.parametrize("ctas", ["2", "4"])
+def test_in_place_scan_with_clusters(monkeypatch, ctas):
+    """state_in == state_out with several CTAs per head: every CTA reads the
+    initial state before rank 0 writes the final one into the same buffer."""
+    monkeypatch.setenv("GDN_TC_CTAS", ctas)
+    wl = inputs.Workload("inplace_scan", 1, 6, 64, 3, 256, "bf16", 532, "l2", "rollout")
+    assert gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D) == (gdn.KERNEL_TC, int(ctas))
+    q, k, v, g, be = device_workload(wl)
+    m0 = torch.from_numpy(inputs.state(wl)).cuda()
+    ref_o, ref_s = gdn.frame_scan(q, k, v, g, be, m0.clone())
+    st = m0.clone()
+    o, _ = gdn.frame_scan(q, k, v, g, be, st, state_out=st)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert torch.equal(o, ref_o) and torch.equal(st, ref_s)

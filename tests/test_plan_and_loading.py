@@ -11,7 +11,7 @@ import torch
 from frame_wise_gated_scan_b200 import build, gdn
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-TC, SIMT = gdn.KERNEL_TC, gdn.KERNEL_SIMT
+TC, SIMT, STEP = gdn.KERNEL_TC, gdn.KERNEL_SIMT, gdn.KERNEL_STEP
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -33,14 +33,26 @@ def test_plan_without_a_device(monkeypatch):
 
 def test_plan_rules_that_hold_on_any_machine(monkeypatch):
     monkeypatch.delenv("GDN_TC_CTAS", raising=False)
-    assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)          # a single frame: one CTA per head
+    monkeypatch.delenv("GDN_STEP_CTAS", raising=False)
+    # a single frame: the row-split kernel, 4 CTAs per head share the rows
+    assert gdn.plan(1, 32, 1, 880, 64) == (STEP, 4)
+    assert gdn.plan(4, 16, 1, 1536, 64) == (STEP, 4)       # 384 rows per CTA, its limit
+    assert gdn.plan(1, 32, 1, 1537, 64) == (TC, 1)         # more rows: one CTA streams them
+    assert gdn.plan(1, 2, 1, 1, 64) == (STEP, 4)
+    assert gdn.plan(1, 2, 1, 64, 128) == (SIMT, 1)         # D = 128 single frame: CUDA cores
+    monkeypatch.setenv("GDN_STEP_CTAS", "2")
+    assert gdn.plan(1, 32, 1, 500, 64) == (STEP, 2)
+    assert gdn.plan(1, 32, 1, 880, 64) == (STEP, 4)        # 440 rows per CTA would not fit
+    monkeypatch.setenv("GDN_STEP_CTAS", "0")               # off: the scan kernel, one CTA
+    assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)
+    monkeypatch.delenv("GDN_STEP_CTAS")
     assert gdn.plan(4, 16, 241, 1350, 128) == (SIMT, 1)    # D = 128: CUDA-core kernel
     assert gdn.plan(1, 2, 8, 64, 32) == (SIMT, 1)          # D = 32
     for forced in ("1", "2", "4"):
         monkeypatch.setenv("GDN_TC_CTAS", forced)
         assert gdn.plan(1, 32, 961, 880, 64) == (TC, int(forced))
     monkeypatch.setenv("GDN_TC_CTAS", "3")                 # not a cluster size it builds
-    assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)
+    assert gdn.plan(1, 32, 2, 880, 64) == (TC, 4) or gdn.plan(1, 32, 2, 880, 64)[0] == TC
     with pytest.raises(gdn.GdnError):
         gdn.plan(1, 32, 961, 880, 48)
 

@@ -43,6 +43,12 @@ def test_noalloc_limit_is_checked_on_the_host():
     # within the limit the ordinary argument checks apply
     assert L.gdn_frame_scan_noalloc(None, *fake[1:], 1, MAX_HEADS, 4, 64, 64,
                                     None) == GDN_ERR_NULL
+    # the argument checks come before the limit
+    assert L.gdn_frame_scan_noalloc(None, *fake[1:], 3, 11, 4, 64, 64, None) == GDN_ERR_NULL
+    # a plan without the ring (one frame: the row-split single-frame kernel) has
+    # no limit; the NULL q stops the call before any launch
+    assert gdn.plan(4, 50, 1, 64, 64)[0] == gdn.KERNEL_STEP
+    assert L.gdn_frame_scan_noalloc(None, *fake[1:], 4, 50, 1, 64, 64, None) == GDN_ERR_NULL
 
 
 @pytest.mark.gpu
