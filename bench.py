@@ -1,14 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the frame-wise GDN scan (libgdn) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload rollout] [--impl libgdn|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libgdn|reference]
 
-One step is one gdn_frame_scan over the whole workload (every head, every
-frame) with the inputs already resident in HBM. The inputs (10.4 GB for the
-961-frame rollout) are far larger than L2, so no L2 flush is needed between
-steps. With N > 1 (torchrun) every rank scans its own copy of the workload on
-its own GPU: the heads are independent, there is no collective on the data
-path, and the scaling is weak. Rank 0 prints one JSON line.
+One step is one gdn_frame_scan over the whole 961-frame rollout (32 heads of
+961 frames of 880 tokens, D = 64, bf16) with the inputs already resident in
+HBM. The inputs (10.4 GB) are far larger than L2, so no L2 flush is needed
+between steps. With N > 1 (torchrun) every rank scans its own copy of the
+workload on its own GPU: the heads are independent, there is no collective on
+the data path, and the scaling is weak. Rank 0 prints one JSON line.
+
+After the timed region the same line gains, each timed with CUDA events on
+the launching stream:
+  step_latency   961 gdn_frame_step calls carrying the state in place (the
+                 chunk-causal rollout), per-call p50/p99, and the final state's
+                 distance to the scan's;
+  workloads      the short clip and the stress batch through gdn_frame_scan,
+                 and the causal temporal conv on the rollout's shapes, each with
+                 its throughput and HBM roofline fraction;
+  e2e            the headline through frame_scan_host on pinned host buffers;
+  cpu_baseline   the float64 oracle on the host's cores.
 
 --impl reference times the float64 CPU oracle (the only reference this
 method has) on a bounded sample of the same workload, rank 0 only.
@@ -50,8 +61,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--frames", type=int, default=0,
                     help="run only the first N frames of the workload (profiling captures)")
-    ap.add_argument("--step-calls", type=int, default=200,
+    ap.add_argument("--step-calls", type=int, default=961,
                     help="gdn_frame_step calls timed one by one for the step latency (0: skip)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the short, stress and conv workloads (profiling captures)")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="timed launches of each extra workload")
     return ap.parse_args()
 
 
@@ -62,6 +77,9 @@ def dist_env():
     return rank, world, local
 
 
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, the peak the GDN task quotes
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -69,6 +87,16 @@ def measured_peaks():
             p = json.load(f)
         return float(p["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def roofline(alg_bytes, launch_s, traffic=None):
+    """HBM roofline record for one launch of `alg_bytes` algorithmic bytes."""
+    peak, kind = measured_peaks()
+    achieved = alg_bytes / launch_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": kind, "traffic": traffic,
+            "frac_nominal": achieved / NOMINAL_HBM_GBS, "peak_nominal": NOMINAL_HBM_GBS,
+            "algorithmic_bytes_per_launch": alg_bytes}
 
 
 def _strip_comments(src: str) -> str:
@@ -162,54 +190,58 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
 
 
-def device_inputs(wl, device):
-    import torch
-    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    shape = (wl.B, wl.H, wl.T, wl.S, wl.D)
-    q = torch.empty(shape, dtype=dt, device=device)
-    k = torch.empty_like(q)
-    v = torch.empty_like(q)
-    g = torch.empty((wl.B, wl.H, wl.T), dtype=torch.float32, device=device)
-    be = torch.empty_like(g)
-    for b, h, qq, kk, vv, gg, bb in inputs.iter_heads_packed(wl):
-        for dst, src in ((q, qq), (k, kk), (v, vv)):
-            t = torch.from_numpy(src.view(np.int16)).view(torch.bfloat16) if wl.dtype == "bf16" \
-                else torch.from_numpy(src)
-            dst[b, h].copy_(t)
-        g[b, h].copy_(torch.from_numpy(gg))
-        be[b, h].copy_(torch.from_numpy(bb))
-    return q, k, v, g, be
+def _oracle_head_job(args):
+    """One head of the workload through the float64 oracle (pool worker)."""
+    wl, b, h, T = args
+    from oracle import gdn_scan_ref
+    q, k, v, g, be = inputs.head(wl, b, h, T)
+    t0 = time.perf_counter()
+    gdn_scan_ref(q, k, v, g, be)
+    return time.perf_counter() - t0
 
 
 def cpu_baseline(wl, seconds: float):
-    """The float64 oracle, as it stands, on whole heads of the workload until
-    the time budget is spent (at least one head's first frames)."""
-    from oracle import gdn_scan_ref
+    """The float64 oracle, as it stands, on the host's cores: heads of the
+    workload run in parallel, one per process of a spawn-started pool of
+    os.cpu_count() processes, each over the first frames of its head, until
+    about `seconds` of wall time is spent. Each process runs BLAS single-threaded
+    (OMP/OPENBLAS/MKL_NUM_THREADS=1), so the cores go to heads, not to small
+    matrix products."""
+    import multiprocessing as mp
+    cores = os.cpu_count() or 1
+    chunk = min(wl.T, 24)
+    env_keys = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+    saved = {k: os.environ.get(k) for k in env_keys}
+    for k in env_keys:
+        os.environ[k] = "1"
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        cores = 1
-    done_frames = 0
-    heads = 0
-    t_total = 0.0
-    chunk = min(wl.T, 64)
-    b = h = 0
-    while t_total < seconds:
-        T = min(chunk, wl.T)
-        q, k, v, g, be = inputs.head(wl, b, h, T)
-        t0 = time.perf_counter()
-        gdn_scan_ref(q, k, v, g, be)
-        t_total += time.perf_counter() - t0
-        done_frames += T
-        heads += 1
-        h = (h + 1) % wl.H
-        if h == 0:
-            b = (b + 1) % wl.B
-    return {"value": done_frames / t_total, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{heads} runs of the float64 oracle over the first {chunk} frames of one "
-                      f"head each (S={wl.S}, D={wl.D}), {t_total:.1f} s of CPU time; "
-                      f"numpy BLAS threads={cores}"}
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(cores) as pool:
+            pool.map(_oracle_head_job, [(wl, 0, 0, 1)] * cores)      # start-up, imports
+            heads_done, oracle_s, t0 = 0, 0.0, time.perf_counter()
+            while True:
+                batch = [(wl, (i // wl.H) % wl.B, i % wl.H, chunk)
+                         for i in range(heads_done, heads_done + cores)]
+                oracle_s += sum(pool.map(_oracle_head_job, batch))
+                heads_done += cores
+                if time.perf_counter() - t0 >= seconds:
+                    break
+            wall = time.perf_counter() - t0
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    frames = heads_done * chunk
+    # Each process times its oracle calls alone (its inputs are drawn outside
+    # that time); all cores run heads at once, so the rate is frames over the
+    # oracle time per core.
+    return {"value": frames / (oracle_s / cores), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads_done} head runs of the float64 oracle over the first {chunk} frames "
+                      f"of a head (S={wl.S}, D={wl.D}), {cores} at a time in a pool of {cores} "
+                      f"processes, BLAS single-threaded; {oracle_s:.1f} s of oracle time over "
+                      f"{wall:.1f} s of wall time"}
 
 
 def run_reference(args, wl):
@@ -249,6 +281,69 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def _time_launches(fn, n, stream, warmup=3):
+    """Mean device time of `fn` (one launch each), CUDA events on `stream`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / n
+
+
+KERNEL_NAMES = {1: "simt", 2: "tcgen05", 3: "tcgen05 row-split (single frame)"}
+
+
+def scan_workload(name, device, stream, n):
+    """One extra GDN workload through gdn_frame_scan: throughput and roofline."""
+    import torch
+    from frame_wise_gated_scan_b200 import gdn
+    wl = inputs.WORKLOADS[name]
+    q, k, v, g, be = inputs.device_draw(wl, device)
+    out = torch.empty_like(q)
+    st = torch.empty((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
+    launch_s = _time_launches(lambda: gdn.frame_scan(q, k, v, g, be, None, out=out, state_out=st),
+                              n, stream)
+    if gdn.device_status() != 0:
+        raise RuntimeError(f"a device-side wait ran out in the {name} workload")
+    kern, ctas = gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D)
+    rec = {"config": {"B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T, "S": wl.S},
+           "kernel": KERNEL_NAMES[kern], "ctas_per_head": ctas, "launches": n,
+           "ms_per_launch": launch_s * 1e3, "value": wl.heads * wl.T / launch_s, "unit": UNIT,
+           "gflops": inputs.flops(wl) / launch_s / 1e9,
+           "roofline": roofline(inputs.algorithmic_bytes(wl), launch_s, recorded_traffic(name)),
+           "l2": ("inputs larger than L2, no flush" if 3 * q.numel() * q.element_size() > 126e6
+                  else "inputs fit in L2: launches run warm, back to back")}
+    del q, k, v, out
+    return rec
+
+
+def conv_workload(device, stream, n):
+    """The causal temporal conv on the rollout's shapes: throughput and roofline."""
+    import torch
+    from frame_wise_gated_scan_b200 import gdn
+    wl = inputs.CONV_WORKLOADS["conv_rollout"]
+    x, w, bias, cache = inputs.conv_device_draw(wl, device)
+    y = torch.empty_like(x)
+    c_out = torch.empty_like(cache)
+    launch_s = _time_launches(
+        lambda: gdn.temporal_conv(x, w, bias, cache, frames_per_block=wl.F, y=y, cache_out=c_out),
+        n, stream)
+    rec = {"config": {"B": wl.B, "T": wl.T, "S": wl.S, "C": wl.C, "frames_per_block": wl.F},
+           "kernel": "cuda cores, 16-byte streams", "launches": n,
+           "ms_per_launch": launch_s * 1e3,
+           "value": wl.B * wl.T * wl.S / launch_s, "unit": "tokens/s",
+           "roofline": roofline(inputs.conv_bytes(wl), launch_s),
+           "l2": "inputs larger than L2 (3.5 GB read per launch), no flush"}
+    del x, y
+    return rec
+
+
 def main():
     args = parse()
     wl = inputs.WORKLOADS[args.workload]
@@ -272,7 +367,7 @@ def main():
     torch.cuda.set_device(device)
 
     kern, ctas = gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D)
-    q, k, v, g, be = device_inputs(wl, device)
+    q, k, v, g, be = inputs.device_draw(wl, device)
     out = torch.empty_like(q)
     st = torch.empty((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
@@ -312,11 +407,11 @@ def main():
     value = multi.whole_job_rate(units, args.steps, world, max_ms)
     mean_launch_s = statistics.mean(launch_ms) / 1e3
     alg_bytes = inputs.algorithmic_bytes(wl)
-    achieved = alg_bytes / mean_launch_s / 1e9
-    peak, peak_kind = measured_peaks()
+    roof = roofline(alg_bytes, mean_launch_s, recorded_traffic(wl.name))
 
-    # Chunk-causal rollout, one gdn_frame_step per frame with the state carried in
-    # place (the "step" workload): per-call latency, after the timed region.
+    # Chunk-causal rollout: one gdn_frame_step per frame with the state carried
+    # in place (the "step" workload), per-call latency, and the final state
+    # against the scan's over the same frames.
     step_lat = None
     if args.step_calls > 0:
         n = min(args.step_calls, wl.T)
@@ -343,15 +438,38 @@ def main():
         dev_us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
         host_us.sort()
         pct = lambda xs, p: xs[min(len(xs) - 1, int(round(p / 100 * (len(xs) - 1))))]
+        # the same frames back to back, no host round trip between calls
+        s_step.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for t in range(n):
+            gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        b2b_us = e0.elapsed_time(e1) * 1e3 / n
+        state_vs_scan = None
+        if n == wl.T:
+            state_vs_scan = float((s_step - st).norm() / st.norm())
+        step_bytes = inputs.algorithmic_bytes(wl, 1) + wl.heads * wl.D * wl.D * 4
         step_lat = {"calls": n, "unit": "us",
                     "device_p50": pct(dev_us, 50), "device_p99": pct(dev_us, 99),
                     "host_p50": pct(host_us, 50), "host_p99": pct(host_us, 99),
+                    "back_to_back_us_per_call": b2b_us,
                     # q, k, v read, out written, gates, the state read and written
-                    "bytes_per_call": inputs.algorithmic_bytes(wl, 1) + wl.heads * wl.D * wl.D * 4,
-                    "kernel": {1: "simt", 2: "tcgen05"}[step_kern], "ctas_per_head": step_ctas,
+                    "bytes_per_call": step_bytes,
+                    "roofline_p50": roofline(step_bytes, pct(dev_us, 50) / 1e6),
+                    "final_state_rel_diff_vs_scan": state_vs_scan,
+                    "kernel": KERNEL_NAMES[step_kern], "ctas_per_head": step_ctas,
                     "how": "device: CUDA events around each call on its stream; host: call "
-                           "plus synchronize, wall clock"}
+                           "plus synchronize, wall clock; back to back: one event pair around "
+                           "all calls"}
         del frames
+
+    extras = None
+    if not args.no_extras and rank == 0:
+        extras = {"short": scan_workload("short", device, stream, args.extra_steps * 10),
+                  "stress": scan_workload("stress", device, stream, args.extra_steps),
+                  "conv": conv_workload(device, stream, args.extra_steps)}
 
     # End to end through the public API on pinned host buffers.
     e2e = None
@@ -388,22 +506,20 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; rollout recipe: Q,V ~ N(0,1), K rows L2-normalised, "
-                "gamma ~ U(.95,1), beta ~ U(.2,1))",
+        "data": "synthetic (seeded on the device; rollout recipe: Q,V ~ N(0,1), K rows "
+                "L2-normalised, gamma ~ U(.95,1), beta ~ U(.2,1))",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T, "S": wl.S,
                    "global_batch": wl.B * world, "seq_len": wl.T * wl.S,
                    "parallelism": f"replicas x{world} (heads independent, no collective)",
-                   "kernel": {1: "simt", 2: "tcgen05"}[kern], "ctas_per_head": ctas,
+                   "kernel": KERNEL_NAMES[kern], "ctas_per_head": ctas,
                    "l2": "inputs larger than L2 (10.4 GB read per step), no flush"},
         "gpu_launches": args.steps,
-        "hbm_gbs": achieved,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": recorded_traffic(wl.name),
-                     "algorithmic_bytes_per_launch": alg_bytes},
+        "hbm_gbs": roof["achieved"],
+        "roofline": roof,
         "clocks": clocks.summary(),
         "e2e": e2e,
         "step_latency": step_lat,
+        "workloads": extras,
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)

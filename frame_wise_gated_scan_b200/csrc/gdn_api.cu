@@ -50,6 +50,11 @@ int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
     *ctas = step;
     return GDN_KERNEL_STEP;
   }
+  const int tc128 = (f == GDN_KERNEL_SIMT) ? 0 : gdn::tc128_ctas_per_head(B, H, T, S, D);
+  if (tc128 > 0) {
+    *ctas = tc128;
+    return GDN_KERNEL_TC;
+  }
   const int tc = (f == GDN_KERNEL_SIMT) ? 0 : gdn::tc_ctas_per_head(B, H, T, S, D);
   if (tc > 0) {
     *ctas = tc;
@@ -80,8 +85,9 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   int ctas = 1;
   const int kern = elt_bytes == 4 ? GDN_KERNEL_SIMT : choose_kernel(B, H, T, S, D, &ctas);
   // The fixed scratch of the no-alloc call holds the transition-operand ring,
-  // which only the tensor-core kernel with more than one CTA per head uses.
-  if (noalloc && kern == GDN_KERNEL_TC && ctas > 1 && (long long)B * H > GDN_NOALLOC_MAX_HEADS)
+  // which only the D = 64 tensor-core kernel with more than one CTA per head uses.
+  if (noalloc && kern == GDN_KERNEL_TC && D == 64 && ctas > 1 &&
+      (long long)B * H > GDN_NOALLOC_MAX_HEADS)
     return GDN_ERR_SCRATCH;
 
   gdn::Problem p;
@@ -110,6 +116,8 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
       err = gdn::launch_step_bf16(p, ctas);   // allocates nothing
     else if (kern != GDN_KERNEL_TC)
       err = gdn::launch_simt_bf16(p);   // allocates nothing either way
+    else if (D == 128)
+      err = gdn::launch_tc128_bf16(p);        // allocates nothing
     else
       err = noalloc ? gdn::launch_tc_bf16_noalloc(p, ctas) : gdn::launch_tc_bf16(p, ctas);
   }
@@ -205,6 +213,21 @@ int gdn_temporal_conv(const void* x, const float* w, const float* bias, const vo
   p.F = frames_per_block;
   p.stream = static_cast<cudaStream_t>(stream);
   return gdn::launch_tconv_bf16(p) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_rope3d(const void* x, void* y, int B, int H, int T, int S, int D, int grid_w, int t0,
+               void* stream) {
+  const int sz = check_sizes(B, H, T, S, D);
+  if (sz != GDN_OK) return sz;
+  if (grid_w < 1 || t0 < 0 || (long long)t0 + T > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (!x || !y) return GDN_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(y, 16)) return GDN_ERR_ALIGN;
+  const size_t n = (size_t)B * H * T * S * D * 2;
+  if (x != y && overlap(x, n, y, n)) return GDN_ERR_ALIAS;
+  return gdn::launch_rope_bf16(x, y, B, H, T, S, D, grid_w, t0, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GDN_OK
+             : GDN_ERR_CUDA;
 }
 
 int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head) {

@@ -37,6 +37,11 @@ cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head);
 // GDN_NOALLOC_MAX_HEADS; calls that overlap on the GPU race on the array.
 cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head);
 
+// tcgen05 kernel for D = 128 (gdn_tc128.cu): a cluster of two CTAs per head,
+// producer and reader. Returns 2 if it takes these sizes, else 0.
+int tc128_ctas_per_head(int B, int H, int T, int S, int D);
+cudaError_t launch_tc128_bf16(const Problem& p);
+
 // Row-split single-frame kernel (gdn_step.cu): T = 1, D = 64, a cluster of
 // CTAs per head sharing the frame's rows. Returns the CTAs per head for these
 // sizes, or 0 if it does not take them.
@@ -55,6 +60,12 @@ struct ConvProblem {
   cudaStream_t stream;
 };
 cudaError_t launch_tconv_bf16(const ConvProblem& p);
+
+// 3D RoPE (gdn_rope.cu; the rotation itself is in gdn_rope.cuh).
+struct RopeParams;
+void rope_params(RopeParams* rp, int D, int grid_w, int t0);
+cudaError_t launch_rope_bf16(const void* x, void* y, int B, int H, int T, int S, int D, int grid_w,
+                             int t0, cudaStream_t stream);
 
 // Host helpers (gdn_host.cu).
 // TMA map of a [frames][S][D] bf16 array as the 3-D tensor (D, S, frames),

@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = i
         L.gdn_temporal_conv.argtypes = [vp, fp, fp, vp, vp, vp, i, i, i, i, i, vp]
         L.gdn_temporal_conv.restype = i
+        L.gdn_rope3d.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
+        L.gdn_rope3d.restype = i
         L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
         L.gdn_plan.restype = i
         L.gdn_device_status.argtypes = []
@@ -248,6 +250,26 @@ def temporal_conv(x, w, bias=None, cache_in=None, *, frames_per_block=None, y=No
     if st != 0:
         raise GdnError(st, "gdn_temporal_conv")
     return y, cache_out
+
+
+def rope3d(x, grid_w, t0=0, *, out=None):
+    """3D RoPE of queries or keys (gdn_rope3d): x [B,H,T,S,D] bf16 CUDA tensor,
+    token r of a frame at grid row r // grid_w, column r % grid_w, frame index
+    t0 + tau. out may be x (in place). Returns the rotated tensor."""
+    if x.dim() != 5 or x.dtype != torch.bfloat16 or x.device.type != "cuda":
+        raise ValueError("x must be a [B,H,T,S,D] bfloat16 CUDA tensor")
+    B, H, T, S, D = x.shape
+    _check(x, "x", torch.bfloat16, x.shape, x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _check(out, "out", torch.bfloat16, x.shape, x.device)
+    with torch.cuda.device(x.device):
+        st = lib().gdn_rope3d(_ptr(x), _ptr(out), B, H, T, S, D, int(grid_w), int(t0),
+                              _stream_handle(x.device))
+    if st != 0:
+        raise GdnError(st, "gdn_rope3d")
+    return out
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,

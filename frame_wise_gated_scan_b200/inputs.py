@@ -259,3 +259,58 @@ def conv_bytes(wl: ConvWorkload) -> int:
     and bias, the cache read and written."""
     n = wl.B * wl.T * wl.S * wl.C
     return 2 * n * 2 + wl.C * 16 + 2 * wl.B * wl.S * wl.C * 2
+
+
+# ---- device-side draws for timing runs. Seeded and with the workloads'
+# distributions, but a different stream from the per-frame generators above:
+# the parity tests use those; only the benchmark uses these (kernel time does
+# not depend on the values).
+
+def device_draw(wl: Workload, device, seed_offset: int = 0):
+    """q, k, v [B,H,T,S,D] (bf16 or fp32) and gamma, beta [B,H,T] fp32 drawn
+    on `device` with torch's generator, following the workload's recipe."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1_000_003 * wl.seed + seed_offset)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    shape = (wl.B, wl.H, wl.T, wl.S, wl.D)
+
+    def normal(*shp):
+        return torch.randn(shp, generator=gen, device=device, dtype=torch.float32)
+
+    def uniform(lo, hi, shp):
+        return lo + (hi - lo) * torch.rand(shp, generator=gen, device=device, dtype=torch.float32)
+
+    q = normal(*shape).to(dt)
+    k = normal(*shape)
+    if wl.key_mode in ("l2", "lognormal"):
+        k = k / k.norm(dim=-1, keepdim=True)
+    if wl.key_mode == "lognormal":
+        k = k * torch.exp(normal(*shape[:-1], 1))
+    k = k.to(dt)
+    v = normal(*shape).to(dt)
+    gs = (wl.B, wl.H, wl.T)
+    if wl.gate_mode == "tiny":
+        g, b = uniform(0.85, 1.0, gs), uniform(0.0, 1.0, gs)
+    elif wl.gate_mode == "short":
+        g, b = torch.sigmoid(3.0 + 0.5 * normal(*gs)), torch.sigmoid(normal(*gs))
+    elif wl.gate_mode == "rollout":
+        g, b = uniform(0.95, 1.0, gs), uniform(0.2, 1.0, gs)
+    elif wl.gate_mode == "stress":
+        g, b = uniform(0.99, 1.0, gs), torch.ones(gs, device=device)
+    else:
+        raise ValueError(wl.gate_mode)
+    return q, k, v, g.contiguous(), b.contiguous()
+
+
+def conv_device_draw(wl: ConvWorkload, device):
+    """x [B,T,S,C] bf16, taps w [C,3], bias [C] fp32 and a cache [B,S,C] bf16,
+    drawn on `device` with torch's generator (same distributions as above)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1_000_003 * wl.seed)
+    x = torch.randn((wl.B, wl.T, wl.S, wl.C), generator=gen, device=device).to(torch.bfloat16)
+    w = torch.randn((wl.C, 3), generator=gen, device=device) / math.sqrt(3.0)
+    bias = 0.1 * torch.randn((wl.C,), generator=gen, device=device)
+    cache = torch.randn((wl.B, wl.S, wl.C), generator=gen, device=device).to(torch.bfloat16)
+    return x, w, bias, cache

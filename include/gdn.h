@@ -75,12 +75,17 @@ typedef enum gdn_status {
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
- * Arithmetic (D = 64, tensor-core kernel): K^T K and K^T V accumulate in fp32
- * on tcgen05 tensor cores; the state M is kept in fp32 on chip across all T
- * frames and updated as M <- gamma M + A' M + c in fp32 registers, where the
- * product A' M (A' = -gamma beta s^2 K^T K) and the read-out Q M take M and
- * A' rounded to bf16 with fp32 accumulation; out is rounded to bf16 (round
- * to nearest even). D = 32 and 128 run the update in fp32 on CUDA cores.
+ * Arithmetic (D = 64 and 128, tensor-core kernels): K^T K and K^T V
+ * accumulate in fp32 on tcgen05 tensor cores; the state M is kept in fp32 on
+ * chip across all T frames and updated as M <- gamma M + A' M + c in fp32,
+ * where the product A' M (A' = -gamma beta s^2 K^T K; at D = 128 it is
+ * accumulated onto K^T V before the scale beta s) and the read-out Q M take M
+ * and A' rounded to bf16 with fp32 accumulation; out is rounded to bf16
+ * (round to nearest even). D = 64 runs a cluster of 1, 2 or 4 CTAs per head
+ * (gdn_plan); D = 128 a cluster of two, one streaming K and V and running the
+ * recurrence, one streaming Q and writing out. A single frame at D = 64 runs
+ * the row-split kernel of gdn_frame_step. D = 32 runs the update in fp32 on
+ * CUDA cores.
  * On the seeded rollout workload the per-frame relative error against a
  * float64 reference is about 2.4e-3 for out and 2e-6 for the final state. */
 GDN_API int gdn_frame_scan(const void* q, const void* k, const void* v,
@@ -213,6 +218,24 @@ GDN_API int gdn_frame_step_f32_ex(const float* q, const float* k, const float* v
 GDN_API int gdn_temporal_conv(const void* x, const float* w, const float* bias,
                               const void* cache_in, void* cache_out, void* y,
                               int B, int T, int S, int C, int frames_per_block, void* stream);
+
+/* 3D rotary position embedding of queries or keys, applied before the scan
+ * ("SANA-Video" ICLR 2026 oral transcript, shadowingenglish.com: 3D RoPE for
+ * the linear attention). The talk gives no layout; this library's reading:
+ * the head dimension D is cut into contiguous sections for the frame axis t,
+ * the grid-row axis h and the grid-column axis w, of 2*floor(D/6) dims for h
+ * and for w and the rest for t (D = 64: 24 + 20 + 20; D = 128: 44 + 42 + 42).
+ * Inside a section of D_a dims, dims (2i, 2i+1) form pair i and turn
+ * counter-clockwise by p * 10000^(-2i / D_a), p the token's position on that
+ * axis: t0 + tau for the tau-th frame of the call, and for token r of a frame
+ * on a grid grid_w tokens wide, h = r / grid_w and w = r % grid_w.
+ *
+ * x, y: [B][H][T][S][D] bf16, 16-byte aligned; y may equal x (in place), else
+ * they must not overlap. The angle is p * freq in fp32 (freq from double),
+ * cos and sin by sincosf, the rotation in fp32, y rounded to bf16 (nearest
+ * even). D in {32, 64, 128}; grid_w >= 1; t0 >= 0. Allocates nothing. */
+GDN_API int gdn_rope3d(const void* x, void* y, int B, int H, int T, int S, int D, int grid_w,
+                       int t0, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
  * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head

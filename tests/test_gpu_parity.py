@@ -125,15 +125,23 @@ def test_step_chain_rollout_matches_scan():
 
 @pytest.mark.slow
 def test_stress_full_size_sampled_heads():
+    """The stress workload (B=4, H=16, D=128, T=241, S=1350) on the D = 128
+    tensor-core kernel, in the launch bench.py times; sampled heads against the
+    oracle, every output finite."""
     wl = inputs.WORKLOADS["stress"]
+    assert gdn.plan(wl.B, wl.H, wl.T, wl.S, wl.D) == (gdn.KERNEL_TC, 2)
     q, k, v, g, be = workload_on_device("stress")
     out, st = gdn.frame_scan(q, k, v, g, be)
     torch.cuda.synchronize()
     assert gdn.device_status() == 0
     assert torch.isfinite(out).all() and torch.isfinite(st).all(), "stress: NaN/Inf"
-    for b, h in [(0, 0), (3, 15)]:
+    worst = (0.0, 0.0)
+    for b, h in [(0, 0), (1, 7), (3, 15)]:
         ro, rs = oracle_head(wl, b, h)
-        assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16, f"stress b{b} h{h}")
+        eo, es = assert_close(to_np64(out[b, h]), ro, to_np64(st[b, h]), rs, TOL_BF16,
+                              f"stress b{b} h{h}")
+        worst = (max(worst[0], eo), max(worst[1], es))
+    print(f"stress full size: worst per-frame out error {worst[0]:.3e}, state {worst[1]:.3e}")
 
 
 def test_null_state_means_zero_and_state_out_optional():
@@ -190,7 +198,7 @@ def test_bf16_no_delta_tensor_core(monkeypatch, ctas):
     _scan_and_compare(wl, state_in=inputs.state(wl, scale=0.5), delta=False)
 
 
-@pytest.mark.parametrize("D", [32, 128])
+@pytest.mark.parametrize("D", [32])
 def test_bf16_no_delta_cuda_cores(D):
     wl = inputs.Workload(f"nodelta_d{D}", 1, 2, D, 5, 130, "bf16", 510 + D, "gauss", "tiny")
     _scan_and_compare(wl, state_in=inputs.state(wl, scale=0.5), delta=False)

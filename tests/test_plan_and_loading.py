@@ -39,14 +39,14 @@ def test_plan_rules_that_hold_on_any_machine(monkeypatch):
     assert gdn.plan(4, 16, 1, 1536, 64) == (STEP, 4)       # 384 rows per CTA, its limit
     assert gdn.plan(1, 32, 1, 1537, 64) == (TC, 1)         # more rows: one CTA streams them
     assert gdn.plan(1, 2, 1, 1, 64) == (STEP, 4)
-    assert gdn.plan(1, 2, 1, 64, 128) == (SIMT, 1)         # D = 128 single frame: CUDA cores
+    assert gdn.plan(1, 2, 1, 64, 128) == (TC, 2)           # D = 128: producer + reader CTAs
     monkeypatch.setenv("GDN_STEP_CTAS", "2")
     assert gdn.plan(1, 32, 1, 500, 64) == (STEP, 2)
     assert gdn.plan(1, 32, 1, 880, 64) == (STEP, 4)        # 440 rows per CTA would not fit
     monkeypatch.setenv("GDN_STEP_CTAS", "0")               # off: the scan kernel, one CTA
     assert gdn.plan(1, 32, 1, 880, 64) == (TC, 1)
     monkeypatch.delenv("GDN_STEP_CTAS")
-    assert gdn.plan(4, 16, 241, 1350, 128) == (SIMT, 1)    # D = 128: CUDA-core kernel
+    assert gdn.plan(4, 16, 241, 1350, 128) == (TC, 2)      # D = 128: producer + reader CTAs
     assert gdn.plan(1, 2, 8, 64, 32) == (SIMT, 1)          # D = 32
     for forced in ("1", "2", "4"):
         monkeypatch.setenv("GDN_TC_CTAS", forced)
