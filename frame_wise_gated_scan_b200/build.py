@@ -31,22 +31,29 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+DEBUG_LIB = os.path.join(PKG, "libgdn_debug.so")
+
+
 def build(debug: bool = False, verbose: bool = False, force: bool = False,
-          trace_out: str | None = None) -> str:
+          trace_out: str | None = None, out: str | None = None) -> str:
     """Builds libgdn.so. With trace_out, builds instead a pipeline-trace variant
     (GDN_TRACE: per-frame event timestamps of head 0, read with gdn_trace_copy)
-    at that path; the library the binding loads is left untouched."""
-    out = trace_out or LIB
-    if not force and not debug and not trace_out and not needs_build():
-        return LIB
+    at that path; the library the binding loads is left untouched. With
+    debug=True, builds the GDN_DEBUG variant (device-wait budget read from
+    GDN_DEBUG_WAIT_NS) at `out`, by default libgdn_debug.so."""
+    if debug and out is None:
+        out = DEBUG_LIB
+    out = trace_out or out or LIB
+    if not force and not trace_out and not needs_build(out):
+        return out
     cmd = [nvcc(), *ARCH, "-std=c++17", "-O3", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
            "-I", INCLUDE, "-I", CSRC, "-o", out, *sources(), "-lcudart_static", "-ldl", "-lrt",

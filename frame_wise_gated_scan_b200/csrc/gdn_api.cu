@@ -9,6 +9,7 @@
 
 #include "gdn.h"
 #include "gdn_internal.h"
+#include "gdn_rope.cuh"
 
 namespace {
 
@@ -66,7 +67,8 @@ int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
 
 int run(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
         const float* state_in, float* state_out, void* out, int B, int H, int T, int S, int D,
-        void* stream, int elt_bytes, bool noalloc = false, unsigned int flags = 0) {
+        void* stream, int elt_bytes, bool noalloc = false, unsigned int flags = 0,
+        const gdn::RopeParams* rope = nullptr) {
   const int sz = check_sizes(B, H, T, S, D);
   if (sz != GDN_OK) return sz;
   if (flags & ~GDN_FLAG_NO_DELTA) return GDN_ERR_FLAGS;
@@ -84,6 +86,7 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
     return GDN_ERR_ALIAS;
   int ctas = 1;
   const int kern = elt_bytes == 4 ? GDN_KERNEL_SIMT : choose_kernel(B, H, T, S, D, &ctas);
+  if (rope && kern != GDN_KERNEL_STEP) return GDN_ERR_UNSUPPORTED;
   // The fixed scratch of the no-alloc call holds the transition-operand ring,
   // which only the D = 64 tensor-core kernel with more than one CTA per head uses.
   if (noalloc && kern == GDN_KERNEL_TC && D == 64 && ctas > 1 &&
@@ -113,7 +116,7 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
     err = gdn::launch_simt_f32(p);
   } else {
     if (kern == GDN_KERNEL_STEP)
-      err = gdn::launch_step_bf16(p, ctas);   // allocates nothing
+      err = gdn::launch_step_bf16(p, ctas, rope);   // allocates nothing
     else if (kern != GDN_KERNEL_TC)
       err = gdn::launch_simt_bf16(p);   // allocates nothing either way
     else if (D == 128)
@@ -144,6 +147,17 @@ int gdn_frame_step(const void* q, const void* k, const void* v, const float* gam
                    const float* beta, const float* state_in, float* state_out, void* out, int B,
                    int H, int S, int D, void* stream) {
   return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 2);
+}
+
+int gdn_frame_step_rope(const void* q, const void* k, const void* v, const float* gamma,
+                        const float* beta, const float* state_in, float* state_out, void* out,
+                        int B, int H, int S, int D, int grid_w, int frame_index, unsigned int flags,
+                        void* stream) {
+  if (grid_w < 1 || frame_index < 0) return GDN_ERR_SHAPE;
+  gdn::RopeParams rp;
+  gdn::rope_params(&rp, 64, grid_w, frame_index);
+  return run(q, k, v, gamma, beta, state_in, state_out, out, B, H, 1, S, D, stream, 2, false, flags,
+             &rp);
 }
 
 int gdn_frame_scan_f32(const float* q, const float* k, const float* v, const float* gamma,
@@ -258,6 +272,8 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_SCRATCH:
       return "B * H exceeds GDN_NOALLOC_MAX_HEADS (32), the fixed scratch of gdn_frame_scan_noalloc";
     case GDN_ERR_FLAGS: return "flags holds bits other than GDN_FLAG_NO_DELTA";
+    case GDN_ERR_UNSUPPORTED:
+      return "the fused 3D RoPE step takes D = 64 and S <= 1536 (the row-split single-frame kernel)";
     default: return "unknown gdn_status";
   }
 }

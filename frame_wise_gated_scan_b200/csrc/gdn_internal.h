@@ -45,8 +45,10 @@ cudaError_t launch_tc128_bf16(const Problem& p);
 // Row-split single-frame kernel (gdn_step.cu): T = 1, D = 64, a cluster of
 // CTAs per head sharing the frame's rows. Returns the CTAs per head for these
 // sizes, or 0 if it does not take them.
+struct RopeParams;
 int step_ctas_per_head(int B, int H, int T, int S, int D);
-cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head);
+// rope: null, or the 3D RoPE to apply to Q and K in shared memory first.
+cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head, const RopeParams* rope = nullptr);
 
 // Causal temporal convolution (gdn_conv.cu), arrays as documented in include/gdn.h.
 struct ConvProblem {
@@ -62,7 +64,6 @@ struct ConvProblem {
 cudaError_t launch_tconv_bf16(const ConvProblem& p);
 
 // 3D RoPE (gdn_rope.cu; the rotation itself is in gdn_rope.cuh).
-struct RopeParams;
 void rope_params(RopeParams* rp, int D, int grid_w, int t0);
 cudaError_t launch_rope_bf16(const void* x, void* y, int B, int H, int T, int S, int D, int grid_w,
                              int t0, cudaStream_t stream);

@@ -37,6 +37,7 @@
 
 #include "gdn.h"
 #include "gdn_internal.h"
+#include "gdn_rope.cuh"
 #include "gdn_wait.cuh"
 #include "sm100_ptx.h"
 
@@ -100,6 +101,8 @@ struct StepParams {
   float s;        // key scale 1/sqrt(D*S)
   float s2;       // its square
   float delta;    // 1: delta rule; 0: GDN_FLAG_NO_DELTA (A' = 0)
+  int rope;       // 1: rotate Q and K by 3D RoPE in shared memory before use
+  RopeParams rp;  // its layout; rp.t0 is the frame's absolute index
 };
 
 __device__ __forceinline__ float bf16_round(float x) {
@@ -190,6 +193,29 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   cluster_sync();   // every CTA's barriers are initialised and armed
   const uint32_t tmem = ld_shared_u32(sb + kOffTmemPtr);
   bool issued_mma = false;
+
+  // ---------------------------------------------------------------- 1b. 3D RoPE (optional)
+  // Q and K turned in place once they land, before any MMA reads them. The
+  // swizzle only permutes whole 16-byte chunks of a row, and a chunk holds 4
+  // whole pairs: physical chunk c of local row rho is logical chunk c ^ (rho & 7).
+  if (p.rope && nbox > 0) {
+    const bool kv_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad);
+    const bool q_ok = warp_wait(bar(kBarQ), 0, ctl, kStLoad);
+    if (kv_ok && q_ok) {
+      const int nchunks = nbox * kBox * 8;
+      for (int e = threadIdx.x; e < 2 * nchunks; e += kThreads) {
+        const int which = e / nchunks;             // 0: K, 1: Q
+        const int ce = e - which * nchunks;
+        const int rho = ce >> 3, cp = ce & 7;
+        const uint32_t addr = sb + (which ? kOffQ : kOffK) + (uint32_t)rho * 128u + (uint32_t)cp * 16u;
+        uint4 v = ld_shared_u4(addr);
+        rope_chunk(p.rp, p.rp.t0, r0 + rho, cp ^ (rho & 7), v);
+        st_shared_v4(addr, v);
+      }
+      fence_proxy_async_cta();   // rotated tiles visible to the tensor cores
+    }
+    __syncthreads();
+  }
 
   // ---------------------------------------------------------------- 2. partial K^T [K V]
   if (warp == 1 && lane == 0 && nbox > 0) {
@@ -436,7 +462,7 @@ int chunk_rows(int S, int P) {
 }
 
 template <int P>
-cudaError_t launch_p(const Problem& pr) {
+cudaError_t launch_p(const Problem& pr, const RopeParams* rope) {
   cudaError_t e = prepare<P>();
   if (e != cudaSuccess) return e;
   StepParams p;
@@ -458,6 +484,9 @@ cudaError_t launch_p(const Problem& pr) {
   p.s = pr.key_scale;
   p.s2 = (float)(1.0 / ((double)kD * (double)pr.S));
   p.delta = pr.delta ? 1.f : 0.f;
+  p.rope = rope ? 1 : 0;
+  if (rope) p.rp = *rope;
+  else rope_params(&p.rp, kD, 1, 0);
 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -493,11 +522,11 @@ int step_ctas_per_head(int B, int H, int T, int S, int D) {
   return P;
 }
 
-cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head) {
+cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head, const RopeParams* rope) {
   if (p.T != 1 || p.D != kD) return cudaErrorInvalidValue;
   switch (ctas_per_head) {
-    case 2: return launch_p<2>(p);
-    case 4: return launch_p<4>(p);
+    case 2: return launch_p<2>(p, rope);
+    case 4: return launch_p<4>(p, rope);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -35,7 +35,8 @@
 // ring loader (lane 0) and read-out MMA issuer (lane 16); warps 4-7 recurrence
 // epilogue; 8-11 A'/c epilogue; 12-15 output epilogue.
 //
-// Every wait is bounded (kTimeoutNs). A wait that runs out sets the device
+// Every wait is bounded (1 s; a GDN_DEBUG build reads the bound of role waits
+// from GDN_DEBUG_WAIT_NS, drains keep 1 s). A wait that runs out sets the device
 // status word and an abort flag in every CTA of the cluster; the other roles
 // then stop, in-flight copies and MMAs are drained, and the kernel returns.
 #include <cuda.h>
@@ -86,7 +87,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr uint64_t kTimeoutNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
+constexpr uint64_t kDrainNs = 1000ull * 1000ull * 1000ull;     // 1 s per drain wait
 constexpr int kThreads = 512;
 constexpr int kD = 64;
 constexpr int kTile = 128;                                      // rows per tile
@@ -190,6 +191,7 @@ struct TcParams {
   float* state_out;
   uint16_t* out;           // bf16 bit patterns
   unsigned int* status;
+  unsigned long long timeout_ns;   // bound of every role wait
   // Transition operands shared by the CTAs of a head (P > 1), per head:
   // kRing frames of [A' (bf16, K-major, swizzled) | c^T (fp32)], their ready
   // flags and per-CTA progress.
@@ -248,6 +250,7 @@ struct Ctl {
   uint32_t abort_addr;    // local shared address of the abort flag
   unsigned int* status;
   int P;
+  uint64_t timeout_ns;    // bound of every role wait (1 s in the shipped library)
 };
 
 __device__ __forceinline__ bool aborted(const Ctl& c) {
@@ -274,7 +277,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ct
   while (true) {
     if (mbar_try(bar, parity)) return true;
     if (aborted(c)) return false;
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > c.timeout_ns) {
       raise_abort(c, code);
       return false;
     }
@@ -294,7 +297,7 @@ __device__ __forceinline__ bool poll_bar(uint32_t bar, uint32_t parity, const Ct
       if (mbar_test(bar, parity)) return true;
     }
     if (aborted(c)) return false;
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > c.timeout_ns) {
       raise_abort(c, code);
       return false;
     }
@@ -319,7 +322,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const C
 __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try(bar, parity)) {
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > kDrainNs) {
       atomicOr(c.status, kStDrain);
       return;
     }
@@ -335,7 +338,7 @@ __device__ __forceinline__ bool wait_global_ge(const unsigned long long* ptr,
   while (true) {
     if (ld_acquire_gpu_u64(ptr) >= v) return true;
     if (aborted(c)) return false;
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > c.timeout_ns) {
       raise_abort(c, code);
       return false;
     }
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
   const int r1 = min(p.S, r0 + p.chunk);
   const int nq = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
   const uint32_t tmem_ptr = sb + L::OFF_TMEM_PTR;
-  Ctl ctl{sb + L::OFF_ABORT, p.status, P};
+  Ctl ctl{sb + L::OFF_ABORT, p.status, P, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NKV; ++i) {
@@ -1057,6 +1060,7 @@ cudaError_t launch_p(const Problem& pr, uint8_t* fixed_scratch) {
   p.state_out = pr.state_out;
   p.out = static_cast<uint16_t*>(pr.out);
   p.status = status;
+  p.timeout_ns = wait_budget_ns();
   p.T = pr.T;
   p.S = pr.S;
   p.ntile = (pr.S + kTile - 1) / kTile;

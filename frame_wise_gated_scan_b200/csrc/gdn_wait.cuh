@@ -1,7 +1,9 @@
 // Bounded waits and the abort protocol shared by the cluster kernels.
 //
 // Every wait on an mbarrier, a peer or a flag gives up after `timeout_ns`
-// (1 s in the shipped library). A wait that runs out records its role in the
+// (1 s in the shipped library; a GDN_DEBUG build takes it from the
+// environment so that tests can make waits run out). Drains of copies and
+// MMAs already in flight always keep the full bound, kDrainNs. A wait that runs out records its role in the
 // device status word (read by gdn_device_status) and raises an abort flag in
 // the shared memory of every CTA of the cluster; the other roles see the flag
 // and stop waiting, so every CTA reaches the same exit path, drains what is
@@ -16,6 +18,8 @@ namespace gdn {
 namespace wait {
 
 using namespace ptx;
+
+constexpr unsigned long long kDrainNs = 1000ull * 1000ull * 1000ull;   // 1 s
 
 struct Ctl {
   uint32_t abort_addr;            // local shared address of the abort flag
@@ -64,12 +68,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const C
   return ok != 0;
 }
 
-// Bounded wait that ignores the abort flag (draining copies and MMAs in flight).
+// Bounded wait that ignores the abort flag (draining copies and MMAs in
+// flight); its bound is kDrainNs whatever the role-wait budget.
 __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Ctl& c,
                                           uint32_t code) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try(bar, parity)) {
-    if (globaltimer_ns() - t0 > c.timeout_ns) {
+    if (globaltimer_ns() - t0 > kDrainNs) {
       atomicOr(c.status, code);
       return;
     }

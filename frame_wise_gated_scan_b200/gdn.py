@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = i
         L.gdn_temporal_conv.argtypes = [vp, fp, fp, vp, vp, vp, i, i, i, i, i, vp]
         L.gdn_temporal_conv.restype = i
+        L.gdn_frame_step_rope.argtypes = step_args[:-1] + [i, i, u, vp]
+        L.gdn_frame_step_rope.restype = i
         L.gdn_rope3d.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
         L.gdn_rope3d.restype = i
         L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
@@ -122,7 +124,7 @@ def _check(t, name, dtype, shape, device):
 
 
 def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state,
-          noalloc=False, flags=0):
+          noalloc=False, flags=0, rope=None):
     if q.dim() != (4 if step else 5):
         raise ValueError("q must be [B,H,S,D] for a step, [B,H,T,S,D] for a scan")
     device = q.device
@@ -158,11 +160,17 @@ def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state
     if not step:
         args.append(T)
     args += [S, D]
-    if flags:
+    if rope is not None:
+        if not step or dt != torch.bfloat16:
+            raise ValueError("the fused 3D RoPE is a bf16 single-frame option")
+        args += [int(rope[0]), int(rope[1]), flags]
+    elif flags:
         args.append(flags)
     args.append(_stream_handle(device))
     bf16 = dt == torch.bfloat16
-    if flags:
+    if rope is not None:
+        fn = L.gdn_frame_step_rope
+    elif flags:
         if step:
             fn = L.gdn_frame_step_ex if bf16 else L.gdn_frame_step_f32_ex
         else:
@@ -205,12 +213,13 @@ def frame_scan_noalloc(q, k, v, gamma, beta, state_in=None, *, out, state_out=No
 
 
 def frame_step(q, k, v, gamma, beta, state_in=None, *, out=None, state_out=None,
-               want_state=True, delta=True):
+               want_state=True, delta=True, rope=None):
     """One frame per head (chunk-causal rollout). q, k, v: [B,H,S,D];
     gamma, beta: [B,H]. state_out may be state_in (in-place carry).
-    delta=False as in frame_scan."""
+    delta=False as in frame_scan. rope=(grid_w, frame_index) turns q and k by
+    3D RoPE inside the kernel first (gdn_frame_step_rope)."""
     return _call(True, q, k, v, gamma, beta, state_in, out, state_out, want_state,
-                 flags=0 if delta else FLAG_NO_DELTA)
+                 flags=0 if delta else FLAG_NO_DELTA, rope=rope)
 
 
 def temporal_conv(x, w, bias=None, cache_in=None, *, frames_per_block=None, y=None,

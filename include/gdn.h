@@ -71,7 +71,8 @@ typedef enum gdn_status {
   GDN_ERR_TIMEOUT = -6,         /* a device-side wait ran out (from gdn_device_status) */
   GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
   GDN_ERR_SCRATCH = -8,         /* gdn_frame_scan_noalloc: a ring plan with B * H > GDN_NOALLOC_MAX_HEADS */
-  GDN_ERR_FLAGS = -9            /* unknown bits in `flags` (the _ex calls) */
+  GDN_ERR_FLAGS = -9,           /* unknown bits in `flags` (the _ex calls) */
+  GDN_ERR_UNSUPPORTED = -10     /* gdn_frame_step_rope: sizes its fused kernel does not take */
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
@@ -236,6 +237,20 @@ GDN_API int gdn_temporal_conv(const void* x, const float* w, const float* bias,
  * even). D in {32, 64, 128}; grid_w >= 1; t0 >= 0. Allocates nothing. */
 GDN_API int gdn_rope3d(const void* x, void* y, int B, int H, int T, int S, int D, int grid_w,
                        int t0, void* stream);
+
+/* gdn_frame_step with 3D RoPE fused into its frame load: the row-split kernel
+ * turns the frame's Q and K rows in shared memory as they arrive (the layout
+ * of gdn_rope3d, frame position frame_index, grid grid_w tokens wide), before
+ * any contraction reads them, so the rotated q and k never travel to HBM.
+ * The result equals gdn_rope3d on q and on k followed by gdn_frame_step_ex,
+ * bit for bit. Takes the sizes the row-split kernel takes (gdn_plan reports
+ * GDN_KERNEL_STEP: D = 64, S <= 1536), else GDN_ERR_UNSUPPORTED; flags as in
+ * gdn_frame_step_ex. grid_w >= 1 and frame_index >= 0 (else GDN_ERR_SHAPE). */
+GDN_API int gdn_frame_step_rope(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int S, int D, int grid_w, int frame_index,
+                   unsigned int flags, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
  * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head

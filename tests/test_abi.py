@@ -21,7 +21,7 @@ def test_every_declared_symbol_is_exported(L):
     assert set(names) >= {"gdn_frame_scan", "gdn_frame_step", "gdn_frame_scan_f32",
                           "gdn_frame_step_f32", "gdn_frame_scan_noalloc", "gdn_frame_scan_ex",
                           "gdn_frame_step_ex", "gdn_frame_scan_f32_ex", "gdn_frame_step_f32_ex",
-                          "gdn_plan",
+                          "gdn_plan", "gdn_temporal_conv", "gdn_rope3d", "gdn_frame_step_rope",
                           "gdn_device_status",
                           "gdn_status_string", "gdn_version"}
     out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strings(L):
     assert gdn.version() == 10000
-    for st in range(-9, 1):
+    for st in range(-10, 1):
         s = gdn.status_string(st)
         assert s and s != "unknown gdn_status"
     assert gdn.status_string(-99) == "unknown gdn_status"
@@ -99,3 +99,28 @@ def test_plan_is_host_logic(L):
     assert kern == gdn.KERNEL_SIMT and ctas == 1
     with pytest.raises(gdn.GdnError):
         gdn.plan(1, 1, 1, 1, 40)
+
+
+def test_conv_rope_and_fused_step_validate_on_the_host(L):
+    p = ctypes.c_void_p
+    x, y, w = p(0x10000000), p(0x20000000), p(0x30000000)
+    conv = lambda *a, **kw: L.gdn_temporal_conv(*a)
+    assert L.gdn_temporal_conv(x, w, None, None, None, y, 1, 4, 3, 12, 2, None) == -2   # C % 8
+    assert L.gdn_temporal_conv(x, w, None, None, None, y, 1, 4, 3, 16, 0, None) == -2   # F = 0
+    assert L.gdn_temporal_conv(None, w, None, None, None, y, 1, 4, 3, 16, 2, None) == -1
+    assert L.gdn_temporal_conv(p(0x10000008), w, None, None, None, y, 1, 4, 3, 16, 2, None) == -4
+    assert L.gdn_temporal_conv(x, w, None, None, None, p(0x10000000 + 64), 1, 4, 3, 16, 2,
+                               None) == -7                                           # y overlaps x
+    assert L.gdn_temporal_conv(x, w, None, p(0x40000000), p(0x40000000 + 16), y, 1, 4, 3, 16, 2,
+                               None) == -7                                           # caches overlap
+    assert L.gdn_rope3d(x, y, 1, 1, 2, 8, 64, 0, 0, None) == -2                       # grid_w = 0
+    assert L.gdn_rope3d(x, y, 1, 1, 2, 8, 64, 4, -1, None) == -2                      # t0 < 0
+    assert L.gdn_rope3d(x, y, 1, 1, 2, 8, 48, 4, 0, None) == -3
+    assert L.gdn_rope3d(None, y, 1, 1, 2, 8, 64, 4, 0, None) == -1
+    assert L.gdn_rope3d(x, p(0x10000000 + 32), 1, 1, 2, 8, 64, 4, 0, None) == -7
+    args = [p(0x1000000), p(0x2000000), p(0x3000000), p(0x4000000), p(0x5000000), None, None,
+            p(0x6000000)]
+    assert L.gdn_frame_step_rope(*args, 1, 2, 64, 128, 8, 0, 0, None) == -10          # D = 128
+    assert L.gdn_frame_step_rope(*args, 1, 2, 2000, 64, 8, 0, 0, None) == -10         # S too large
+    assert L.gdn_frame_step_rope(*args, 1, 2, 64, 64, 0, 0, 0, None) == -2            # grid_w = 0
+    assert L.gdn_frame_step_rope(*args, 1, 2, 64, 64, 8, 0, 2, None) == -9            # flags
