@@ -160,6 +160,55 @@ int gdn_frame_step_rope(const void* q, const void* k, const void* v, const float
              &rp);
 }
 
+int gdn_frame_stream(const void* q, const void* k, const void* v, const float* gamma,
+                     const float* beta, const float* state_in, float* state_out, void* out, int B,
+                     int H, int S, int D, int ring, const unsigned long long* posted,
+                     unsigned long long* done, unsigned int* slot_counters,
+                     unsigned long long idle_timeout_ns, unsigned int flags, void* stream) {
+  const int sz = check_sizes(B, H, 1, S, D);
+  if (sz != GDN_OK) return sz;
+  if (ring < 1 || (long long)ring * B * H > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (flags & ~GDN_FLAG_NO_DELTA) return GDN_ERR_FLAGS;
+  if (!q || !k || !v || !gamma || !beta || !out || !posted || !done || !slot_counters)
+    return GDN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(gamma, 4) ||
+      !aligned(beta, 4) || !aligned(posted, 8) || !aligned(done, 8) || !aligned(slot_counters, 4))
+    return GDN_ERR_ALIGN;
+  const size_t n = (size_t)ring * B * H * S * D * 2;
+  const size_t ns = (size_t)B * H * D * D * sizeof(float);
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) ||
+      overlap(out, n, state_in, ns) || overlap(out, n, state_out, ns))
+    return GDN_ERR_ALIAS;
+  if (state_in && state_out && state_in != state_out && overlap(state_in, ns, state_out, ns))
+    return GDN_ERR_ALIAS;
+  if (!gdn::stream_supported(B, H, S, D)) return GDN_ERR_UNSUPPORTED;
+  gdn::Problem p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gamma = gamma;
+  p.beta = beta;
+  p.state_in = state_in;
+  p.state_out = state_out;
+  p.out = out;
+  p.B = B;
+  p.H = H;
+  p.T = 1;
+  p.S = S;
+  p.D = D;
+  p.key_scale = (float)(1.0 / sqrt((double)D * (double)S));
+  p.delta = (flags & GDN_FLAG_NO_DELTA) == 0;
+  p.stream = static_cast<cudaStream_t>(stream);
+  gdn::StreamQueue qd;
+  qd.posted = posted;
+  qd.done = done;
+  qd.slot_counters = slot_counters;
+  qd.ring = ring;
+  qd.idle_timeout_ns = idle_timeout_ns;
+  return gdn::launch_stream_bf16(p, qd, nullptr) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 int gdn_frame_scan_f32(const float* q, const float* k, const float* v, const float* gamma,
                        const float* beta, const float* state_in, float* state_out, float* out,
                        int B, int H, int T, int S, int D, void* stream) {
@@ -273,7 +322,8 @@ const char* gdn_status_string(int status) {
       return "B * H exceeds GDN_NOALLOC_MAX_HEADS (32), the fixed scratch of gdn_frame_scan_noalloc";
     case GDN_ERR_FLAGS: return "flags holds bits other than GDN_FLAG_NO_DELTA";
     case GDN_ERR_UNSUPPORTED:
-      return "the fused 3D RoPE step takes D = 64 and S <= 1536 (the row-split single-frame kernel)";
+      return "sizes the call's kernel does not take (gdn_frame_step_rope: D = 64, S <= 1536; "
+             "gdn_frame_stream: the same, with every head's cluster resident at once)";
     default: return "unknown gdn_status";
   }
 }

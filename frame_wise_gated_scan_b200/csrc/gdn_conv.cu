@@ -14,7 +14,7 @@
 // with no contraction, so it runs on CUDA cores with 16-byte accesses. Thread
 // (column, segment) owns 8 channels of one token (one 16-byte vector per
 // frame) over a run of frames, keeps the previous, current and next frame in
-// registers, and keeps four frames of loads in flight. Warps read and write
+// registers, and keeps eight frames of loads in flight. Warps read and write
 // 512 contiguous bytes per frame. Segments split long runs of frames across
 // threads so that small S * C still fills the GPU; a segment reads the frame
 // before it (or the cache) once.
@@ -27,7 +27,7 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kAhead = 4;   // frames loaded ahead of the one being written
+constexpr int kAhead = 8;   // frames loaded ahead of the one being written
 
 __device__ __forceinline__ void unpack8(const uint4 r, float* f) {
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
@@ -65,7 +65,7 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   return pol;
 }
 
-__global__ void __launch_bounds__(kThreads) gdn_tconv_kernel(
+__global__ void __launch_bounds__(kThreads, 2) gdn_tconv_kernel(
     const uint4* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     const uint4* cache_in, uint4* cache_out, uint4* __restrict__ y, int T, int S, int C8, int F,
     int seg_frames, int nseg, long long cols) {

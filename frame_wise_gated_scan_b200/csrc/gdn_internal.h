@@ -49,6 +49,20 @@ struct RopeParams;
 int step_ctas_per_head(int B, int H, int T, int S, int D);
 // rope: null, or the 3D RoPE to apply to Q and K in shared memory first.
 cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head, const RopeParams* rope = nullptr);
+// Frame queue of the persistent streaming launch (gdn_frame_stream).
+struct StreamQueue {
+  const unsigned long long* posted;   // host-mapped, device view
+  unsigned long long* done;           // host-mapped, device view
+  unsigned int* slot_counters;        // device [ring], zero
+  int ring;
+  unsigned long long idle_timeout_ns;
+};
+// 1 if the streaming kernel takes these sizes (D = 64, S <= 1536 and every
+// head's cluster resident at once), else 0.
+int stream_supported(int B, int H, int S, int D);
+// p.q/k/v/out are rings [ring][B][H][S][D], p.gamma/beta rings [ring][B][H];
+// p.T is unused.
+cudaError_t launch_stream_bf16(const Problem& p, const StreamQueue& q, const RopeParams* rope);
 
 // Causal temporal convolution (gdn_conv.cu), arrays as documented in include/gdn.h.
 struct ConvProblem {

@@ -62,17 +62,18 @@ constexpr uint32_t kOffQ = 2 * kRegion;
 constexpr uint32_t kOffM0 = 3 * kRegion;          // M (fp32, 64 x 64), 16 KB
 constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (64/P rows) x 512 B
 constexpr uint32_t kOffMg = kOffRed + 32768;      // M' in bf16: 64 rows x 128 B, 128-byte swizzle
-constexpr uint32_t kOffBar = kOffMg + 8192;
+constexpr uint32_t kOffM0r = kOffMg + 8192;       // M rounded to bf16, as fp32, 16 KB
+constexpr uint32_t kOffBar = kOffM0r + 16384;
 enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarGather, kBarO, kBarDrain, kNumBars };
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
+constexpr uint32_t kOffGo = kOffAbort + 4;         // streaming: the verdict of the wait for a frame
 constexpr uint32_t kBytes = kOffAbort + 16;
 constexpr uint32_t kSmemAlloc = kBytes + 1024;    // base alignment slack
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0, "swizzled regions are 1 KB aligned");
 
 // Regions reused once the partial product has read K (K region) and V (V region):
-constexpr uint32_t kOffM0r = kOffK;               // M rounded to bf16, as fp32, 16 KB
 constexpr uint32_t kOffArow = kOffK + 16384;      // A' rows (fp32 holding bf16 values), <= 8 KB
 constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
 constexpr uint32_t kOffMst = kOffK + 32768;       // own rows of M' in bf16, <= 4 KB
@@ -82,8 +83,17 @@ constexpr uint32_t kOffOut = kOffV;               // output tiles, 3 x 16 KB (af
 // Status bits (shared with the scan kernel's numbering scheme, high bits).
 enum : uint32_t {
   kStLoad = 1u << 16, kStMma = 1u << 17, kStRed = 1u << 18, kStGather = 1u << 19,
-  kStOut = 1u << 20, kStDrain = 1u << 21, kStConfig = 1u << 22
+  kStOut = 1u << 20, kStDrain = 1u << 21, kStConfig = 1u << 22, kStIdle = 1u << 23
 };
+
+__device__ __forceinline__ unsigned long long ld_acquire_sys_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_sys_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 struct StepParams {
   CUtensorMap tm_q;
@@ -102,7 +112,14 @@ struct StepParams {
   float s2;       // its square
   float delta;    // 1: delta rule; 0: GDN_FLAG_NO_DELTA (A' = 0)
   int rope;       // 1: rotate Q and K by 3D RoPE in shared memory before use
-  RopeParams rp;  // its layout; rp.t0 is the frame's absolute index
+  RopeParams rp;  // its layout; rp.t0 is the (first) frame's absolute index
+  // frame queue (streaming launch only)
+  const unsigned long long* posted;   // host-mapped: frames posted; bit 63 set: stop after them
+  unsigned long long* done;           // host-mapped: frames every head has completed
+  unsigned int* frame_done;           // device [ring]: CTAs done with the frame in each slot (0 at start)
+  int ring;                           // frame slots
+  int heads;                          // B * H
+  unsigned long long idle_ns;         // bound of the wait for the next frame
 };
 
 __device__ __forceinline__ float bf16_round(float x) {
@@ -121,7 +138,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int P>
+// kStream = false: one frame (gdn_frame_step). kStream = true: a persistent
+// launch that serves frames from a ring of slots as the host posts them (the
+// frame queue of gdn_frame_stream), keeping the state on chip between frames.
+template <int P, bool kStream>
 __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_constant__ StepParams p) {
   constexpr int R = kD / P;   // state rows this CTA updates
   static_assert(R % 16 == 0, "a warp's 16 rows go to one CTA");
@@ -148,31 +168,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   const int nq = (nrows + 127) / 128;   // 128-row read-out tiles
   auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * i; };
   Ctl ctl{sb + kOffAbort, p.status, p.timeout_ns, P};
-  const float g = __ldg(p.gamma + bh);
-  const float be = __ldg(p.beta + bh);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
-    // The exchange barriers are armed before the cluster barrier below, and
-    // peers only send after it.
-    mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
-    mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
-    if (nbox > 0) {
-      const uint64_t pol = policy_evict_first();   // read once
-      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
-      for (int b = 0; b < nbox; ++b) {
-        tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, bh, pol);
-        tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, bh, pol);
-      }
-      mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
-      for (int b = 0; b < nbox; ++b)
-        tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, bh, pol);
-    }
   }
-  // The initial state, whole, in every CTA. It is read here, before the first
-  // cluster barrier, and the final state is written only after it: so
+  // The initial state, whole, in every CTA, with its bf16 rounding (the
+  // operand of the product A' M). It is read here, before the first cluster
+  // barrier, and the final state is written only after it: so
   // state_in == state_out is safe.
   {
     const float4* src = reinterpret_cast<const float4*>(p.state_in + (size_t)bh * kD * kD);
@@ -180,6 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       const float4 x = p.state_in ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
       asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kOffM0 + 16u * i),
                    "f"(x.x), "f"(x.y), "f"(x.z), "f"(x.w)
+                   : "memory");
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kOffM0r + 16u * i),
+                   "f"(bf16_round(x.x)), "f"(bf16_round(x.y)), "f"(bf16_round(x.z)),
+                   "f"(bf16_round(x.w))
                    : "memory");
     }
   }
@@ -190,227 +198,347 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();   // every CTA's barriers are initialised and armed
+  cluster_sync();   // every CTA's barriers are initialised
   const uint32_t tmem = ld_shared_u32(sb + kOffTmemPtr);
   bool issued_mma = false;
+  int last = -1;          // the last frame started (its barrier phases may be in flight)
+  bool loads_issued = false;
 
-  // ---------------------------------------------------------------- 1b. 3D RoPE (optional)
-  // Q and K turned in place once they land, before any MMA reads them. The
-  // swizzle only permutes whole 16-byte chunks of a row, and a chunk holds 4
-  // whole pairs: physical chunk c of local row rho is logical chunk c ^ (rho & 7).
-  if (p.rope && nbox > 0) {
-    const bool kv_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad);
-    const bool q_ok = warp_wait(bar(kBarQ), 0, ctl, kStLoad);
-    if (kv_ok && q_ok) {
-      const int nchunks = nbox * kBox * 8;
-      for (int e = threadIdx.x; e < 2 * nchunks; e += kThreads) {
-        const int which = e / nchunks;             // 0: K, 1: Q
-        const int ce = e - which * nchunks;
-        const int rho = ce >> 3, cp = ce & 7;
-        const uint32_t addr = sb + (which ? kOffQ : kOffK) + (uint32_t)rho * 128u + (uint32_t)cp * 16u;
-        uint4 v = ld_shared_u4(addr);
-        rope_chunk(p.rp, p.rp.t0, r0 + rho, cp ^ (rho & 7), v);
-        st_shared_v4(addr, v);
-      }
-      fence_proxy_async_cta();   // rotated tiles visible to the tensor cores
-    }
-    __syncthreads();
-  }
-
-  // ---------------------------------------------------------------- 2. partial K^T [K V]
-  if (warp == 1 && lane == 0 && nbox > 0) {
-    if (wait_bar(bar(kBarKv), 0, ctl, kStLoad)) {
-      tc_fence_after();
-      // A = K^T (M = 64 key dims, one 128-byte atom), B = [K V] (N = 128: the K
-      // and V regions are its two atoms, kRegion apart); both MN-major views of
-      // the row-major tiles; 16 rows per MMA.
-      constexpr uint32_t idesc = idesc_bf16(64, 128, 1, 1);
-      for (int kk = 0; kk < 2 * nbox; ++kk) {
-        const uint64_t a = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
-        const uint64_t b = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
-        mma_bf16(tmem, a, b, idesc, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(bar(kBarMma));
-      issued_mma = true;
-    }
-  }
-
-  // ---------------------------------------------------------------- 3. reduce-scatter
-  // With M = 64 the accumulator row i (key dim) sits in TMEM lane 32(i/16) + i%16:
-  // warp w (< 4) reads lanes 32w.., and its lanes 0-15 hold key rows 16w..16w+15,
-  // columns 0-63 = K^T K, 64-127 = K^T V. Those 16 rows (8 KB of fp32) go to the
-  // CTA that updates them, staged with chunk c of row i at chunk c ^ (i & 7).
-  if (warp < 4) {
-    const bool ok = nbox == 0 || warp_wait(bar(kBarMma), 0, ctl, kStMma);
-    if (ok) {
-      tc_fence_after();
-      const int il = lane & 15;
-      const uint32_t row_addr = sb + kOffSend + (uint32_t)(warp * 16 + il) * 512u;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t v[64];
-        if (nbox > 0) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r16[16];
-            tmem_ld16(tmem + 64 * h + 16 * c + ((uint32_t)(warp * 32) << 16), r16);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
-          }
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) v[e] = 0u;
+  for (int n = 0;; ++n) {
+    const uint32_t ph = (uint32_t)(n & 1);   // phase parity of every per-frame barrier
+    int frame = bh;                          // index along the tensors' frame axis
+    if (kStream) {
+      // ------------------------------------------------------------ 0. next frame or stop
+      if (threadIdx.x == 0) {
+        uint32_t go = 0;
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+          const unsigned long long v = ld_acquire_sys_u64(p.posted);
+          if ((v & ~(1ull << 63)) > (unsigned long long)n) { go = 1; break; }
+          if (v >> 63) break;                                   // stop after the posted frames
+          if (aborted(ctl)) break;
+          if (globaltimer_ns() - t0 > p.idle_ns) { raise_abort(ctl, kStIdle); break; }
+          __nanosleep(256);
         }
-        if (lane < 16) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t cc = 16 * h + c;
-            st_shared_v4(row_addr + ((cc ^ (uint32_t)(il & 7)) << 4),
-                         make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
-          }
-        }
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + kOffGo), "r"(go) : "memory");
       }
-      tc_fence_before();
-      fence_proxy_async_cta();   // staged rows visible to the bulk copy
-      __syncwarp();
-      if (lane == 0) {
-        const uint32_t dst = (uint32_t)(warp * P / 4);
-        const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
-        bulk_copy_to_cluster(mapa(sb + kOffRed + slot_row * 512u, dst),
-                             sb + kOffSend + (uint32_t)warp * 16u * 512u, 16u * 512u,
-                             mapa(bar(kBarRed), dst));
-      }
+      __syncthreads();
+      if (ld_shared_u32(sb + kOffGo) == 0 || aborted(ctl)) break;
+      frame = (n % p.ring) * p.heads + bh;
+    } else if (n > 0) {
+      break;
     }
-  }
+    last = n;
+    const float g = __ldg(p.gamma + frame);
+    const float be = __ldg(p.beta + frame);
 
-  // ---------------------------------------------------------------- 4. recurrence, own rows
-  const bool red_ok = warp_wait(bar(kBarRed), 0, ctl, kStRed);
-  __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
-  if (red_ok && !aborted(ctl)) {
-    const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 K^T K (0 without delta)
-    const float cbs = be * p.s;                    // c = beta s K^T V
-    for (int e = threadIdx.x; e < R * 128; e += kThreads) {
-      const int il = e >> 7, n = e & 127;
-      const uint32_t off = (uint32_t)((((n >> 2) ^ (il & 7)) << 4) + (n & 3) * 4);
-      float sum = 0.f;
-#pragma unroll
-      for (int src = 0; src < P; ++src)
-        sum += ld_shared_f32(sb + kOffRed + (uint32_t)(src * R + il) * 512u + off);
-      if (n < kD)
-        st_shared_f32(sb + kOffArow + (uint32_t)(il * kD + n) * 4u, bf16_round(coef * sum));
-      else
-        st_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + n - kD) * 4u, cbs * sum);
-    }
-    for (int e = threadIdx.x; e < kD * kD; e += kThreads)
-      st_shared_f32(sb + kOffM0r + 4u * e, bf16_round(ld_shared_f32(sb + kOffM0 + 4u * e)));
-  }
-  __syncthreads();
-  if (red_ok && !aborted(ctl)) {
-    const int j = threadIdx.x & 63;      // value column
-    const int ib = threadIdx.x >> 6;     // rows ib, ib + 4, ...
-    constexpr int NR = R / 4;
-    float acc[NR];
-#pragma unroll
-    for (int n = 0; n < NR; ++n) acc[n] = 0.f;
-    if (p.delta != 0.f) {
-#pragma unroll 8
-      for (int k = 0; k < kD; ++k) {
-        const float mk = ld_shared_f32(sb + kOffM0r + (uint32_t)(k * kD + j) * 4u);
-#pragma unroll
-        for (int n = 0; n < NR; ++n)
-          acc[n] = fmaf(ld_shared_f32(sb + kOffArow + (uint32_t)((ib + 4 * n) * kD + k) * 4u), mk, acc[n]);
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < NR; ++n) {
-      const int il = ib + 4 * n;
-      const int gi = (int)rank * R + il;
-      const float m0 = ld_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u);
-      const float m1 = fmaf(g, m0, acc[n]) + ld_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + j) * 4u);
-      if (p.state_out) p.state_out[((size_t)bh * kD + gi) * kD + j] = m1;
-      const __nv_bfloat16 hb = __float2bfloat16_rn(m1);
-      st_shared_u16(sb + kOffMst + swz128((uint32_t)il, (uint32_t)(j >> 3)) + (uint32_t)(j & 7) * 2u,
-                    *reinterpret_cast<const uint16_t*>(&hb));
-    }
-  }
-  fence_proxy_async_cta();   // M' rows visible to the bulk copies
-  __syncthreads();
-  // ---------------------------------------------------------------- 5. all-gather of M' (bf16)
-  if (threadIdx.x == 0 && red_ok && !aborted(ctl)) {
-    for (int d = 0; d < P; ++d)
-      bulk_copy_to_cluster(mapa(sb + kOffMg + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
-                           (uint32_t)R * 128u, mapa(bar(kBarGather), (uint32_t)d));
-  }
-
-  // ---------------------------------------------------------------- 6. read-out O = Q M'
-  if (warp == 1 && lane == 0 && nq > 0) {
-    if (wait_bar(bar(kBarGather), 0, ctl, kStGather) && wait_bar(bar(kBarQ), 0, ctl, kStLoad)) {
-      tc_fence_after();
-      constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);   // Q K-major, M' MN-major
-      for (int i = 0; i < nq; ++i) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = smem_desc(sb + kOffQ + i * 16384 + kk * 32, 16, 1024, 2);
-          const uint64_t b = smem_desc(sb + kOffMg + kk * 2048, 8192, 1024, 2);
-          mma_bf16(tmem + 64 * i, a, b, id_o, kk > 0 ? 1u : 0u);
+    // -------------------------------------------------------------- 1. loads of the frame
+    // The exchange barriers are armed here. A peer's data for this frame can
+    // only come after this CTA completed the previous frame's exchanges, so an
+    // early bulk copy finds the barrier in this frame's phase (its byte count
+    // runs ahead of the arming, which the barrier allows).
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
+      mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
+      if (nbox > 0) {
+        const uint64_t pol = policy_evict_first();   // read once
+        mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
+        for (int b = 0; b < nbox; ++b) {
+          tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
+          tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
         }
+        mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
+        for (int b = 0; b < nbox; ++b)
+          tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, frame, pol);
+        loads_issued = true;
       }
-      mma_commit(bar(kBarO));
-      issued_mma = true;
     }
-  }
-  // Output tiles: warps 4g..4g+3 take tiles g, g + 2, ...; lane l of warp
-  // quarter q holds tile row 32q + l.
-  {
-    const int grp = warp >> 2;
-    const int qd = warp & 3;
-    if (grp < nq) {
-      const bool ok = warp_wait(bar(kBarO), 0, ctl, kStOut);
+
+    // -------------------------------------------------------------- 1b. 3D RoPE (optional)
+    // Q and K turned in place once they land, before any MMA reads them. The
+    // swizzle only permutes whole 16-byte chunks of a row, and a chunk holds 4
+    // whole pairs: physical chunk c of local row rho is logical chunk c ^ (rho & 7).
+    if (p.rope && nbox > 0) {
+      const bool kv_ok = warp_wait(bar(kBarKv), ph, ctl, kStLoad);
+      const bool q_ok = warp_wait(bar(kBarQ), ph, ctl, kStLoad);
+      if (kv_ok && q_ok) {
+        const int nchunks = nbox * kBox * 8;
+        for (int e = threadIdx.x; e < 2 * nchunks; e += kThreads) {
+          const int which = e / nchunks;             // 0: K, 1: Q
+          const int ce = e - which * nchunks;
+          const int rho = ce >> 3, cp = ce & 7;
+          const uint32_t addr = sb + (which ? kOffQ : kOffK) + (uint32_t)rho * 128u + (uint32_t)cp * 16u;
+          uint4 v = ld_shared_u4(addr);
+          rope_chunk(p.rp, p.rp.t0 + n, r0 + rho, cp ^ (rho & 7), v);
+          st_shared_v4(addr, v);
+        }
+        fence_proxy_async_cta();   // rotated tiles visible to the tensor cores
+      }
+      __syncthreads();
+    }
+
+    // -------------------------------------------------------------- 2. partial K^T [K V]
+    if (warp == 1 && lane == 0 && nbox > 0) {
+      if (wait_bar(bar(kBarKv), ph, ctl, kStLoad)) {
+        tc_fence_after();
+        // A = K^T (M = 64 key dims, one 128-byte atom), B = [K V] (N = 128: the K
+        // and V regions are its two atoms, kRegion apart); both MN-major views of
+        // the row-major tiles; 16 rows per MMA.
+        constexpr uint32_t idesc = idesc_bf16(64, 128, 1, 1);
+        for (int kk = 0; kk < 2 * nbox; ++kk) {
+          const uint64_t a = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
+          const uint64_t b = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
+          mma_bf16(tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBarMma));
+        issued_mma = true;
+      }
+    }
+
+    // -------------------------------------------------------------- 3. reduce-scatter
+    // With M = 64 the accumulator row i (key dim) sits in TMEM lane 32(i/16) + i%16:
+    // warp w (< 4) reads lanes 32w.., and its lanes 0-15 hold key rows 16w..16w+15,
+    // columns 0-63 = K^T K, 64-127 = K^T V. Those 16 rows (8 KB of fp32) go to the
+    // CTA that updates them, staged with chunk c of row i at chunk c ^ (i & 7).
+    if (warp < 4) {
+      const bool ok = nbox == 0 || warp_wait(bar(kBarMma), ph, ctl, kStMma);
       if (ok) {
         tc_fence_after();
-        for (int i = grp; i < nq; i += 2) {
+        const int il = lane & 15;
+        const uint32_t row_addr = sb + kOffSend + (uint32_t)(warp * 16 + il) * 512u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
           uint32_t v[64];
+          if (nbox > 0) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r16[16];
-            tmem_ld16(tmem + 64 * i + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r16[16];
+              tmem_ld16(tmem + 64 * h + 16 * c + ((uint32_t)(warp * 32) << 16), r16);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+              for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+            }
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] = 0u;
           }
-          tmem_wait_ld();
-          const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
-          const uint32_t row = (uint32_t)(qd * 32 + lane);
+          if (lane < 16) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-            w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-            w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-            w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-            st_shared_v4(tile + swz128(row, (uint32_t)c), w);
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t cc = 16 * h + c;
+              st_shared_v4(row_addr + ((cc ^ (uint32_t)(il & 7)) << 4),
+                           make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+            }
           }
         }
         tc_fence_before();
-        fence_proxy_async_cta();
-      }
-      named_bar_sync(1 + grp, 128);   // every warp of the group arrives, ok or not
-      if (qd == 0 && lane == 0 && !aborted(ctl)) {
-        const uint64_t pol = policy_evict_first();
-        for (int i = grp; i < nq; i += 2) {
-          const int y0 = r0 + 128 * i;
-          const int y1 = min(r1, y0 + 128);
-          const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
-          for (int y = y0; y < y1; y += kBox)
-            tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, bh, pol);
+        fence_proxy_async_cta();   // staged rows visible to the bulk copy
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t dst = (uint32_t)(warp * P / 4);
+          const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
+          bulk_copy_to_cluster(mapa(sb + kOffRed + slot_row * 512u, dst),
+                               sb + kOffSend + (uint32_t)warp * 16u * 512u, 16u * 512u,
+                               mapa(bar(kBarRed), dst));
         }
-        bulk_commit();
-        bulk_wait0();
+      }
+    }
+
+    // -------------------------------------------------------------- 4. recurrence, own rows
+    const bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed);
+    __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
+    if (red_ok && !aborted(ctl)) {
+      const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 K^T K (0 without delta)
+      const float cbs = be * p.s;                    // c = beta s K^T V
+      for (int e = threadIdx.x; e < R * 128; e += kThreads) {
+        const int il = e >> 7, nn = e & 127;
+        const uint32_t off = (uint32_t)((((nn >> 2) ^ (il & 7)) << 4) + (nn & 3) * 4);
+        float sum = 0.f;
+#pragma unroll
+        for (int src = 0; src < P; ++src)
+          sum += ld_shared_f32(sb + kOffRed + (uint32_t)(src * R + il) * 512u + off);
+        if (nn < kD)
+          st_shared_f32(sb + kOffArow + (uint32_t)(il * kD + nn) * 4u, bf16_round(coef * sum));
+        else
+          st_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + nn - kD) * 4u, cbs * sum);
+      }
+    }
+    __syncthreads();
+    if (red_ok && !aborted(ctl)) {
+      // Thread t updates row il = t / (64 / CPT) of this CTA's rows, value
+      // columns j0 .. j0 + CPT - 1; each k step reads one A' value (shared by
+      // the row's threads) and CPT / 4 float4 of the rounded M row k.
+      constexpr int CPT = R * kD / kThreads;           // 4 (P = 4) or 8 (P = 2)
+      constexpr int TPR = kD / CPT;                    // threads per row
+      const int il = threadIdx.x / TPR;
+      const int j0 = (threadIdx.x % TPR) * CPT;
+      float acc[CPT];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
+      if (p.delta != 0.f) {
+#pragma unroll 4
+        for (int k = 0; k < kD; ++k) {
+          const float a = ld_shared_f32(sb + kOffArow + (uint32_t)(il * kD + k) * 4u);
+#pragma unroll
+          for (int c4 = 0; c4 < CPT / 4; ++c4) {
+            const float4 mk = ld_shared_f4(sb + kOffM0r + (uint32_t)(k * kD + j0 + 4 * c4) * 4u);
+            acc[4 * c4 + 0] = fmaf(a, mk.x, acc[4 * c4 + 0]);
+            acc[4 * c4 + 1] = fmaf(a, mk.y, acc[4 * c4 + 1]);
+            acc[4 * c4 + 2] = fmaf(a, mk.z, acc[4 * c4 + 2]);
+            acc[4 * c4 + 3] = fmaf(a, mk.w, acc[4 * c4 + 3]);
+          }
+        }
+      }
+      const int gi = (int)rank * R + il;
+      float m1[CPT];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        const int j = j0 + c;
+        const float m0 = ld_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u);
+        m1[c] = fmaf(g, m0, acc[c]) + ld_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + j) * 4u);
+        if (kStream) st_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u, m1[c]);   // kept on chip
+      }
+      if (!kStream && p.state_out) {
+        float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)bh * kD + gi) * kD + j0);
+#pragma unroll
+        for (int c4 = 0; c4 < CPT / 4; ++c4)
+          dst[c4] = make_float4(m1[4 * c4], m1[4 * c4 + 1], m1[4 * c4 + 2], m1[4 * c4 + 3]);
+      }
+      // bf16 copy of the row segment, in the swizzled layout of the read-out's
+      // operand: CPT consecutive values sit in one 16-byte chunk (CPT = 8) or
+      // half of one (CPT = 4).
+#pragma unroll
+      for (int c = 0; c < CPT; c += 2) {
+        const int j = j0 + c;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + kOffMst + swz128((uint32_t)il, (uint32_t)(j >> 3)) +
+                                                  (uint32_t)(j & 7) * 2u),
+                     "r"(pack_bf16x2(m1[c], m1[c + 1]))
+                     : "memory");
+      }
+    }
+    fence_proxy_async_cta();   // M' rows visible to the bulk copies
+    __syncthreads();
+    // -------------------------------------------------------------- 5. all-gather of M' (bf16)
+    if (threadIdx.x == 0 && red_ok && !aborted(ctl)) {
+      for (int d = 0; d < P; ++d)
+        bulk_copy_to_cluster(mapa(sb + kOffMg + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
+                             (uint32_t)R * 128u, mapa(bar(kBarGather), (uint32_t)d));
+    }
+
+    // -------------------------------------------------------------- 6. read-out O = Q M'
+    if (warp == 1 && lane == 0 && nq > 0) {
+      if (wait_bar(bar(kBarGather), ph, ctl, kStGather) && wait_bar(bar(kBarQ), ph, ctl, kStLoad)) {
+        tc_fence_after();
+        constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);   // Q K-major, M' MN-major
+        for (int i = 0; i < nq; ++i) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = smem_desc(sb + kOffQ + i * 16384 + kk * 32, 16, 1024, 2);
+            const uint64_t b = smem_desc(sb + kOffMg + kk * 2048, 8192, 1024, 2);
+            mma_bf16(tmem + 64 * i, a, b, id_o, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(bar(kBarO));
+        issued_mma = true;
+      }
+    }
+    // Output tiles: warps 4g..4g+3 take tiles g, g + 2, ...; lane l of warp
+    // quarter q holds tile row 32q + l.
+    {
+      const int grp = warp >> 2;
+      const int qd = warp & 3;
+      if (grp < nq) {
+        const bool ok = warp_wait(bar(kBarO), ph, ctl, kStOut);
+        if (ok) {
+          tc_fence_after();
+          for (int i = grp; i < nq; i += 2) {
+            uint32_t v[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r16[16];
+              tmem_ld16(tmem + 64 * i + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
+            }
+            tmem_wait_ld();
+            const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+            const uint32_t row = (uint32_t)(qd * 32 + lane);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+              w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+              w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+              w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+              st_shared_v4(tile + swz128(row, (uint32_t)c), w);
+            }
+          }
+          tc_fence_before();
+          fence_proxy_async_cta();
+        }
+        named_bar_sync(1 + grp, 128);   // every warp of the group arrives, ok or not
+        if (qd == 0 && lane == 0 && !aborted(ctl)) {
+          const uint64_t pol = policy_evict_first();
+          for (int i = grp; i < nq; i += 2) {
+            const int y0 = r0 + 128 * i;
+            const int y1 = min(r1, y0 + 128);
+            const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+            for (int y = y0; y < y1; y += kBox)
+              tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, frame, pol);
+          }
+          bulk_commit();
+          if (kStream)
+            bulk_wait0();        // the frame is done only once its rows are written
+          else
+            bulk_wait_read0();   // the staging may go once read; the writes finish on their own
+        }
+      }
+    }
+    if (!kStream) continue;
+
+    // -------------------------------------------------------------- 7. frame done (stream)
+    // The next frame's product takes M' in bf16 from the gathered buffer, before
+    // any peer can send the next M' into it (they first need this CTA's next
+    // partial product).
+    {
+      const bool ok = warp_wait(bar(kBarGather), ph, ctl, kStGather);
+      if (ok && !aborted(ctl)) {
+        for (int e = threadIdx.x; e < kD * kD / 2; e += kThreads) {
+          const int row = e >> 5, j = (e & 31) * 2;
+          const uint32_t w = ld_shared_u32(sb + kOffMg + swz128((uint32_t)row, (uint32_t)(j >> 3)) +
+                                          (uint32_t)(j & 7) * 2u);
+          st_shared_f32(sb + kOffM0r + (uint32_t)(row * kD + j) * 4u, __uint_as_float(w << 16));
+          st_shared_f32(sb + kOffM0r + (uint32_t)(row * kD + j + 1) * 4u, __uint_as_float(w & 0xffff0000u));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0 && !aborted(ctl)) {
+      // Every CTA of every head counts itself done with the slot; the last one
+      // resets the count and tells the host.
+      fence_proxy_async_global();
+      __threadfence();
+      const unsigned int total = (unsigned int)(p.heads * P);
+      const unsigned int slot = (unsigned int)(n % p.ring);
+      if (atomicAdd(p.frame_done + slot, 1u) == total - 1u) {
+        p.frame_done[slot] = 0u;
+        __threadfence_system();
+        st_release_sys_u64(p.done, (unsigned long long)(n + 1));
       }
     }
   }
 
   // ---------------------------------------------------------------- exit
+  if (kStream && p.state_out && !aborted(ctl)) {
+    // this CTA's rows of the final state, fp32, kept on chip across the frames
+    for (int e = threadIdx.x; e < R * kD; e += kThreads) {
+      const int gi = (int)rank * R + e / kD;
+      p.state_out[((size_t)bh * kD + gi) * kD + (e % kD)] =
+          ld_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + e % kD) * 4u);
+    }
+  }
   if (warp == 1 && lane == 0 && issued_mma) {   // every MMA done before TMEM is freed
     mma_commit(bar(kBarDrain));
     drain_bar(bar(kBarDrain), 0, ctl, kStDrain);
@@ -422,14 +550,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     // Same verdict in every CTA (the flag is raised in all of them before the
     // raising thread reaches the barrier above). Let copies still in flight
     // land before any CTA of the cluster leaves: loads issued here, and bulk
-    // copies from peers (all issued before that barrier).
-    if (threadIdx.x == 0) {
-      if (nbox > 0) {
-        drain_bar(bar(kBarKv), 0, ctl, kStDrain);
-        drain_bar(bar(kBarQ), 0, ctl, kStDrain);
+    // copies from peers (all issued before that barrier), in the phase of the
+    // last frame started.
+    if (threadIdx.x == 0 && last >= 0) {
+      const uint32_t ph = (uint32_t)(last & 1);
+      if (loads_issued) {
+        drain_bar(bar(kBarKv), ph, ctl, kStDrain);
+        drain_bar(bar(kBarQ), ph, ctl, kStDrain);
       }
-      drain_bar(bar(kBarRed), 0, ctl, kStDrain);
-      drain_bar(bar(kBarGather), 0, ctl, kStDrain);
+      drain_bar(bar(kBarRed), ph, ctl, kStDrain);
+      drain_bar(bar(kBarGather), ph, ctl, kStDrain);
     }
     __syncthreads();
     cluster_sync();
@@ -442,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ host side
 
-template <int P>
+template <int P, bool kStream>
 cudaError_t prepare() {
   static std::atomic<bool> done[64];
   int dev = 0;
@@ -450,7 +580,7 @@ cudaError_t prepare() {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gdn_step_kernel<P>),
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gdn_step_kernel<P, kStream>),
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
   if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
   return e;
@@ -461,46 +591,86 @@ int chunk_rows(int S, int P) {
   return (per + kBox - 1) / kBox * kBox;
 }
 
-template <int P>
-cudaError_t launch_p(const Problem& pr, const RopeParams* rope) {
-  cudaError_t e = prepare<P>();
-  if (e != cudaSuccess) return e;
-  StepParams p;
-  const long long frames = (long long)pr.B * pr.H;
-  if (!make_frame_map(&p.tm_q, pr.q, kD, pr.S, frames, kBox) ||
-      !make_frame_map(&p.tm_k, pr.k, kD, pr.S, frames, kBox) ||
-      !make_frame_map(&p.tm_v, pr.v, kD, pr.S, frames, kBox) ||
-      !make_frame_map(&p.tm_o, pr.out, kD, pr.S, frames, kBox))
-    return cudaErrorInvalidValue;
-  p.status = status_word();
-  if (!p.status) return cudaErrorInvalidDevice;
-  p.gamma = pr.gamma;
-  p.beta = pr.beta;
-  p.state_in = pr.state_in;
-  p.state_out = pr.state_out;
-  p.timeout_ns = wait_budget_ns();
-  p.S = pr.S;
-  p.chunk = chunk_rows(pr.S, P);
-  p.s = pr.key_scale;
-  p.s2 = (float)(1.0 / ((double)kD * (double)pr.S));
-  p.delta = pr.delta ? 1.f : 0.f;
-  p.rope = rope ? 1 : 0;
-  if (rope) p.rp = *rope;
-  else rope_params(&p.rp, kD, 1, 0);
-
+template <int P, bool kStream>
+cudaLaunchConfig_t launch_config(long long heads, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = P;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(frames * P), 1, 1);
+  cfg.gridDim = dim3((unsigned)(heads * P), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemAlloc;
-  cfg.stream = pr.stream;
+  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gdn_step_kernel<P>, p);
+  return cfg;
+}
+
+// Fills the parameters common to both modes; frames = the tensors' frame axis.
+template <int P>
+cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, const RopeParams* rope) {
+  if (!make_frame_map(&p->tm_q, pr.q, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p->tm_k, pr.k, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p->tm_v, pr.v, kD, pr.S, frames, kBox) ||
+      !make_frame_map(&p->tm_o, pr.out, kD, pr.S, frames, kBox))
+    return cudaErrorInvalidValue;
+  p->status = status_word();
+  if (!p->status) return cudaErrorInvalidDevice;
+  p->gamma = pr.gamma;
+  p->beta = pr.beta;
+  p->state_in = pr.state_in;
+  p->state_out = pr.state_out;
+  p->timeout_ns = wait_budget_ns();
+  p->S = pr.S;
+  p->chunk = chunk_rows(pr.S, P);
+  p->s = pr.key_scale;
+  p->s2 = (float)(1.0 / ((double)kD * (double)pr.S));
+  p->delta = pr.delta ? 1.f : 0.f;
+  p->rope = rope ? 1 : 0;
+  if (rope) p->rp = *rope;
+  else rope_params(&p->rp, kD, 1, 0);
+  p->posted = nullptr;
+  p->done = nullptr;
+  p->frame_done = nullptr;
+  p->ring = 1;
+  p->heads = pr.B * pr.H;
+  p->idle_ns = 0;
+  return cudaSuccess;
+}
+
+template <int P>
+cudaError_t launch_p(const Problem& pr, const RopeParams* rope) {
+  cudaError_t e = prepare<P, false>();
+  if (e != cudaSuccess) return e;
+  StepParams p;
+  e = fill_params<P>(&p, pr, (long long)pr.B * pr.H, rope);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config<P, false>((long long)pr.B * pr.H, pr.stream, attr);
+  return cudaLaunchKernelEx(&cfg, gdn_step_kernel<P, false>, p);
+}
+
+// Clusters of the streaming kernel that can be resident at once (every head's
+// cluster must be, since each waits for frames the others complete).
+int stream_resident_clusters() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return -1;
+  }
+  const int known = cache[dev].load(std::memory_order_acquire);
+  if (known != 0) return known - 2;
+  int n = -1;
+  if (prepare<4, true>() == cudaSuccess) {
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = launch_config<4, true>(64, nullptr, attr);
+    if (cudaOccupancyMaxActiveClusters(&n, gdn_step_kernel<4, true>, &cfg) != cudaSuccess) n = -1;
+  }
+  cudaGetLastError();
+  cache[dev].store(n + 2, std::memory_order_release);
+  return n;
 }
 
 }  // namespace
@@ -529,6 +699,29 @@ cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head, const RopePara
     case 4: return launch_p<4>(p, rope);
     default: return cudaErrorInvalidValue;
   }
+}
+
+int stream_supported(int B, int H, int S, int D) {
+  if (D != kD || chunk_rows(S, 4) > kRowsMax) return 0;
+  const int fit = stream_resident_clusters();
+  const long long heads = (long long)B * H;
+  return heads <= (fit >= 0 ? fit : 148 / 4) ? 1 : 0;
+}
+
+cudaError_t launch_stream_bf16(const Problem& pr, const StreamQueue& q, const RopeParams* rope) {
+  cudaError_t e = prepare<4, true>();
+  if (e != cudaSuccess) return e;
+  StepParams p;
+  e = fill_params<4>(&p, pr, (long long)q.ring * pr.B * pr.H, rope);
+  if (e != cudaSuccess) return e;
+  p.posted = q.posted;
+  p.done = q.done;
+  p.frame_done = q.slot_counters;
+  p.ring = q.ring;
+  p.idle_ns = q.idle_timeout_ns;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config<4, true>((long long)pr.B * pr.H, pr.stream, attr);
+  return cudaLaunchKernelEx(&cfg, gdn_step_kernel<4, true>, p);
 }
 
 }  // namespace gdn

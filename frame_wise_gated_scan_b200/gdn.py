@@ -68,6 +68,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_temporal_conv.restype = i
         L.gdn_frame_step_rope.argtypes = step_args[:-1] + [i, i, u, vp]
         L.gdn_frame_step_rope.restype = i
+        ull = ctypes.c_ulonglong
+        L.gdn_frame_stream.argtypes = step_args[:-1] + [i, vp, vp, vp, ull, u, vp]
+        L.gdn_frame_stream.restype = i
         L.gdn_rope3d.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
         L.gdn_rope3d.restype = i
         L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
@@ -279,6 +282,79 @@ def rope3d(x, grid_w, t0=0, *, out=None):
     if st != 0:
         raise GdnError(st, "gdn_rope3d")
     return out
+
+
+class FrameStream:
+    """Chunk-causal streaming through a device-side frame queue
+    (gdn_frame_stream): one persistent launch serves frames as they are
+    posted, keeping the state on chip, with no launch per frame.
+
+    q, k, v, out: [ring, B, H, S, D] bf16 rings and gamma, beta: [ring, B, H]
+    fp32 rings on the device; frame n lives in slot n % ring. Fill a slot
+    (from pinned host memory, or before the launch), then post(); wait(n)
+    returns once frames 0..n-1 are complete. close() stops the kernel and
+    returns the final state. The counters live in pinned host memory.
+    """
+
+    STOP = -(1 << 63)    # bit 63 of the posted counter, as a signed int64
+
+    def __init__(self, q, k, v, gamma, beta, out=None, state_in=None, *, want_state=True,
+                 idle_timeout_s=10.0, delta=True, stream=None):
+        if q.dim() != 5 or q.dtype != torch.bfloat16 or q.device.type != "cuda":
+            raise ValueError("q must be a [ring,B,H,S,D] bfloat16 CUDA tensor")
+        R, B, H, S, D = q.shape
+        dev = q.device
+        for name, t in (("k", k), ("v", v)):
+            _check(t, name, torch.bfloat16, q.shape, dev)
+        _check(gamma, "gamma", torch.float32, (R, B, H), dev)
+        _check(beta, "beta", torch.float32, (R, B, H), dev)
+        if state_in is not None:
+            _check(state_in, "state_in", torch.float32, (B, H, D, D), dev)
+        self.out = torch.empty_like(q) if out is None else out
+        _check(self.out, "out", torch.bfloat16, q.shape, dev)
+        self.state = torch.empty((B, H, D, D), dtype=torch.float32, device=dev) if want_state else None
+        self.counters = torch.zeros(2, dtype=torch.int64, pin_memory=True)   # posted, done
+        self.slots = torch.zeros(R, dtype=torch.int32, device=dev)
+        self.stream = stream or torch.cuda.Stream(dev)
+        self.ring, self.posted = R, 0
+        self._keep = (q, k, v, gamma, beta, state_in)
+        base = self.counters.data_ptr()
+        L = lib()
+        with torch.cuda.device(dev):
+            st = L.gdn_frame_stream(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+                                    _ptr(state_in), _ptr(self.state), _ptr(self.out), B, H, S, D, R,
+                                    ctypes.c_void_p(base), ctypes.c_void_p(base + 8),
+                                    _ptr(self.slots), int(idle_timeout_s * 1e9),
+                                    0 if delta else FLAG_NO_DELTA,
+                                    ctypes.c_void_p(self.stream.cuda_stream))
+        if st != 0:
+            raise GdnError(st, "gdn_frame_stream")
+
+    def post(self, frames=1):
+        """Frames posted so far += frames (their slots must hold their inputs)."""
+        self.posted += frames
+        self.counters[0] = self.posted
+
+    def done(self) -> int:
+        return int(self.counters[1])
+
+    def wait(self, n, timeout_s=10.0):
+        """Polls until frames 0..n-1 are done; returns the time it waited."""
+        import time
+        t0 = time.perf_counter()
+        while int(self.counters[1]) < n:
+            if time.perf_counter() - t0 > timeout_s:
+                raise TimeoutError(f"frame stream: {int(self.counters[1])} of {n} frames done")
+        return time.perf_counter() - t0
+
+    def close(self):
+        """Stops the kernel after the posted frames; returns the final state."""
+        self.counters[0] = self.posted + self.STOP
+        self.stream.synchronize()
+        st = device_status()
+        if st != 0:
+            raise GdnError(st, "gdn_frame_stream")
+        return self.state
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,

@@ -72,7 +72,7 @@ typedef enum gdn_status {
   GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
   GDN_ERR_SCRATCH = -8,         /* gdn_frame_scan_noalloc: a ring plan with B * H > GDN_NOALLOC_MAX_HEADS */
   GDN_ERR_FLAGS = -9,           /* unknown bits in `flags` (the _ex calls) */
-  GDN_ERR_UNSUPPORTED = -10     /* gdn_frame_step_rope: sizes its fused kernel does not take */
+  GDN_ERR_UNSUPPORTED = -10     /* gdn_frame_step_rope, gdn_frame_stream: sizes their kernel does not take */
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
@@ -250,6 +250,47 @@ GDN_API int gdn_frame_step_rope(const void* q, const void* k, const void* v,
                    const float* gamma, const float* beta,
                    const float* state_in, float* state_out, void* out,
                    int B, int H, int S, int D, int grid_w, int frame_index,
+                   unsigned int flags, void* stream);
+
+/* Chunk-causal streaming without a launch per frame: one persistent launch of
+ * the row-split single-frame kernel (gdn_frame_step) serves frames from a
+ * device-side frame queue as they are posted, keeping every head's D x D
+ * state on chip between frames ("NVIDIA Apresenta SANA-WM ...",
+ * acheiumaia.com.br: the chunk-causal autoregressive generator for
+ * sequential rollout; one latent frame per recurrent step, constant state).
+ *
+ * The queue: rings of `ring` frame slots in device memory,
+ *   q, k, v, out   [ring][B][H][S][D] bf16      gamma, beta  [ring][B][H] fp32,
+ * and two counters in host memory mapped into the device (pinned host memory;
+ * pass the device view, which under unified addressing is the host address):
+ *   posted  written by the caller: frames 0 .. posted-1 are in their slots
+ *           (frame n in slot n % ring). Setting bit 63 asks the kernel to stop
+ *           once the posted frames are done.
+ *   done    written by the kernel: frames 0 .. done-1 are complete for every
+ *           head (their out slots are written).
+ * slot_counters: device memory, ring unsigned ints, zero at the call (the
+ * kernel counts the CTAs done with each slot's frame and puts it back to zero).
+ * The caller must fill slot n % ring before posting frame n, and must not
+ * refill a slot before `done` has passed the frame it held. Frames are
+ * processed in order; the state is read from state_in (NULL: zero) at the
+ * start and written to state_out (NULL: not written) when the kernel stops.
+ *
+ * The call enqueues the launch on `stream` and returns; the kernel runs until
+ * stopped. Its wait for the next frame is bounded by idle_timeout_ns: if
+ * neither a frame nor the stop arrives in time it stops early and
+ * gdn_device_status() reports GDN_ERR_TIMEOUT. Only host writes to `posted`
+ * (and copies by the copy engines) may feed it: work on the same GPU that the
+ * caller waits for before posting could find no free SM while the kernel
+ * holds them. Sizes: those of the row-split kernel (D = 64, S <= 1536) with
+ * every head's cluster resident at once (B * H up to about 33 on a B200), else
+ * GDN_ERR_UNSUPPORTED. Update and precision as gdn_frame_step; flags as in
+ * gdn_frame_step_ex. Allocates nothing. */
+GDN_API int gdn_frame_stream(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int S, int D, int ring,
+                   const unsigned long long* posted, unsigned long long* done,
+                   unsigned int* slot_counters, unsigned long long idle_timeout_ns,
                    unsigned int flags, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
