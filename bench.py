@@ -67,6 +67,10 @@ def parse():
                     help="skip the short, stress and conv workloads (profiling captures)")
     ap.add_argument("--extra-steps", type=int, default=20,
                     help="timed launches of each extra workload")
+    ap.add_argument("--extras", default="short,stress,conv,rope",
+                    help="comma-separated extra workloads (short, stress, conv, rope)")
+    ap.add_argument("--extra-frames", type=int, default=0,
+                    help="cut the extra workloads to this many frames (profiling captures)")
     return ap.parse_args()
 
 
@@ -299,11 +303,13 @@ def _time_launches(fn, n, stream, warmup=3):
 KERNEL_NAMES = {1: "simt", 2: "tcgen05", 3: "tcgen05 row-split (single frame)"}
 
 
-def scan_workload(name, device, stream, n):
+def scan_workload(name, device, stream, n, frames=0):
     """One extra GDN workload through gdn_frame_scan: throughput and roofline."""
     import torch
     from frame_wise_gated_scan_b200 import gdn
     wl = inputs.WORKLOADS[name]
+    if frames:
+        wl = wl.with_(T=min(frames, wl.T))
     q, k, v, g, be = inputs.device_draw(wl, device)
     out = torch.empty_like(q)
     st = torch.empty((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
@@ -323,11 +329,13 @@ def scan_workload(name, device, stream, n):
     return rec
 
 
-def conv_workload(device, stream, n):
+def conv_workload(device, stream, n, frames=0):
     """The causal temporal conv on the rollout's shapes: throughput and roofline."""
     import torch
     from frame_wise_gated_scan_b200 import gdn
     wl = inputs.CONV_WORKLOADS["conv_rollout"]
+    if frames:
+        wl = wl.with_(T=min(frames, wl.T))
     x, w, bias, cache = inputs.conv_device_draw(wl, device)
     y = torch.empty_like(x)
     c_out = torch.empty_like(cache)
@@ -341,6 +349,27 @@ def conv_workload(device, stream, n):
            "roofline": roofline(inputs.conv_bytes(wl), launch_s),
            "l2": "inputs larger than L2 (3.5 GB read per launch), no flush"}
     del x, y
+    return rec
+
+
+def rope_workload(device, stream, n, frames=0):
+    """3D RoPE of the rollout's queries (gdn_rope3d, out of place)."""
+    import torch
+    from frame_wise_gated_scan_b200 import gdn
+    wl = inputs.WORKLOADS["rollout"]
+    if frames:
+        wl = wl.with_(T=min(frames, wl.T))
+    q = inputs.device_draw(wl, device, seed_offset=7)[0]
+    y = torch.empty_like(q)
+    launch_s = _time_launches(lambda: gdn.rope3d(q, 40, 0, out=y), n, stream)
+    nbytes = 2 * q.numel() * q.element_size()
+    rec = {"config": {"B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T, "S": wl.S, "grid_w": 40},
+           "kernel": "cuda cores, 16-byte streams", "launches": n,
+           "ms_per_launch": launch_s * 1e3,
+           "value": wl.heads * wl.T * wl.S / launch_s, "unit": "token-rows/s",
+           "roofline": roofline(nbytes, launch_s),
+           "l2": "inputs larger than L2 (3.5 GB read per launch), no flush"}
+    del q, y
     return rec
 
 
@@ -450,11 +479,28 @@ def main():
         state_vs_scan = None
         if n == wl.T:
             state_vs_scan = float((s_step - st).norm() / st.norm())
+        # the same chain captured once as a CUDA graph and replayed: device time
+        # per step without the host's per-call work
+        s_step.zero_()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for t in range(n):
+                gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
+        graph.replay()
+        torch.cuda.synchronize(device)
+        s_step.zero_()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        graph_us = e0.elapsed_time(e1) * 1e3 / n
+        del graph
         step_bytes = inputs.algorithmic_bytes(wl, 1) + wl.heads * wl.D * wl.D * 4
         step_lat = {"calls": n, "unit": "us",
                     "device_p50": pct(dev_us, 50), "device_p99": pct(dev_us, 99),
                     "host_p50": pct(host_us, 50), "host_p99": pct(host_us, 99),
                     "back_to_back_us_per_call": b2b_us,
+                    "graph_us_per_step": graph_us,
                     # q, k, v read, out written, gates, the state read and written
                     "bytes_per_call": step_bytes,
                     "roofline_p50": roofline(step_bytes, pct(dev_us, 50) / 1e6),
@@ -465,11 +511,40 @@ def main():
                            "all calls"}
         del frames
 
+    # The same rollout through the frame queue: one persistent launch, frames
+    # posted one at a time by the host, each timed from post to done.
+    stream_lat = None
+    if args.step_calls > 0:
+        n = min(args.step_calls, wl.T)
+        ring = lambda x: x[:, :, :n].permute(2, 0, 1, *range(3, x.dim())).contiguous()
+        rings = [ring(x) for x in (q, k, v, g, be)]
+        fs = gdn.FrameStream(*rings)
+        lat = []
+        for t in range(n):
+            h0 = time.perf_counter()
+            fs.post()
+            fs.wait(t + 1)
+            lat.append((time.perf_counter() - h0) * 1e6)
+        s_stream = fs.close()
+        lat.sort()
+        pct = lambda xs, p: xs[min(len(xs) - 1, int(round(p / 100 * (len(xs) - 1))))]
+        stream_lat = {"frames": n, "unit": "us", "p50": pct(lat, 50), "p99": pct(lat, 99),
+                      "final_state_rel_diff_vs_scan":
+                          float((s_stream - st).norm() / st.norm()) if n == wl.T else None,
+                      "how": "one gdn_frame_stream launch over the rollout staged as a ring of "
+                             "frame slots; the host posts frame t and polls for it to be done "
+                             "(pinned-memory counters), wall clock per frame"}
+        del rings, fs
+
     extras = None
     if not args.no_extras and rank == 0:
-        extras = {"short": scan_workload("short", device, stream, args.extra_steps * 10),
-                  "stress": scan_workload("stress", device, stream, args.extra_steps),
-                  "conv": conv_workload(device, stream, args.extra_steps)}
+        want = [x.strip() for x in args.extras.split(",") if x.strip()]
+        ef = args.extra_frames
+        run = {"short": lambda: scan_workload("short", device, stream, args.extra_steps * 10, ef),
+               "stress": lambda: scan_workload("stress", device, stream, args.extra_steps, ef),
+               "conv": lambda: conv_workload(device, stream, args.extra_steps, ef),
+               "rope": lambda: rope_workload(device, stream, args.extra_steps, ef)}
+        extras = {name: run[name]() for name in want}
 
     # End to end through the public API on pinned host buffers.
     e2e = None
@@ -519,6 +594,7 @@ def main():
         "clocks": clocks.summary(),
         "e2e": e2e,
         "step_latency": step_lat,
+        "stream_latency": stream_lat,
         "workloads": extras,
     }
     if not args.no_cpu_baseline:

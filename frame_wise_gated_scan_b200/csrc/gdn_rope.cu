@@ -14,21 +14,35 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__global__ void __launch_bounds__(kThreads) gdn_rope_kernel(const uint4* x, uint4* y, long long chunks,
+// One block per frame: cos/sin tables of the frame first (shared memory),
+// then the frame's rows, one 16-byte chunk per thread and step. Frames whose
+// tables would not fit take sincosf per pair instead.
+__global__ void __launch_bounds__(kThreads) gdn_rope_kernel(const uint4* x, uint4* y, long long frames,
                                                             int T, int S, int D8,
                                                             const __grid_constant__ RopeParams rp) {
-  for (long long idx = (long long)blockIdx.x * kThreads + threadIdx.x; idx < chunks;
-       idx += (long long)gridDim.x * kThreads) {
-    const int chunk = (int)(idx % D8);
-    const long long row = idx / D8;
-    const int r = (int)(row % S);
-    const int t = (int)((row / S) % T);
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(x + idx));
-    rope_chunk(rp, rp.t0 + t, r, chunk, v);
-    y[idx] = v;
+  __shared__ float tab[kRopeTabMaxFloats];
+  const int nh = (S - 1) / rp.grid_w + 1;
+  const bool use_tab = rope_tab_floats(rp, nh) <= kRopeTabMaxFloats;
+  const long long chunks = (long long)S * D8;
+  for (long long f = blockIdx.x; f < frames; f += gridDim.x) {
+    const int t = rp.t0 + (int)(f % T);
+    if (use_tab) rope_tab_build(rp, tab, t, 0, nh);
+    const uint4* xs = x + f * chunks;
+    uint4* ys = y + f * chunks;
+    for (long long idx = threadIdx.x; idx < chunks; idx += kThreads) {
+      const int chunk = (int)(idx % D8);
+      const int r = (int)(idx / D8);
+      uint4 v;
+      asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "l"(xs + idx));
+      if (use_tab)
+        rope_chunk_tab(rp, tab, 0, nh, r, chunk, v);
+      else
+        rope_chunk(rp, t, r, chunk, v);
+      ys[idx] = v;
+    }
+    __syncthreads();   // the next frame's table may replace this one
   }
 }
 
@@ -39,6 +53,7 @@ void rope_params(RopeParams* rp, int D, int grid_w, int t0) {
   const int dt = D - 2 * dh;
   rp->nt = dt / 2;
   rp->nth = dt / 2 + dh / 2;
+  rp->np = D / 2;
   rp->grid_w = grid_w;
   rp->t0 = t0;
   for (int i = 0; i < kRopeMaxPairs; ++i) {
@@ -56,14 +71,14 @@ cudaError_t launch_rope_bf16(const void* x, void* y, int B, int H, int T, int S,
                              int t0, cudaStream_t stream) {
   RopeParams rp;
   rope_params(&rp, D, grid_w, t0);
-  const long long chunks = (long long)B * H * T * S * (D / 8);
+  const long long frames = (long long)B * H * T;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long long blocks = (chunks + kThreads - 1) / kThreads;
-  const long long cap = (long long)sms * 32;
+  long long blocks = frames;
+  const long long cap = (long long)sms * 16;
   if (blocks > cap) blocks = cap;
   gdn_rope_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(y), chunks, T, S, D / 8, rp);
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), frames, T, S, D / 8, rp);
   return cudaGetLastError();
 }
 

@@ -63,7 +63,8 @@ constexpr uint32_t kOffM0 = 3 * kRegion;          // M (fp32, 64 x 64), 16 KB
 constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (64/P rows) x 512 B
 constexpr uint32_t kOffMg = kOffRed + 32768;      // M' in bf16: 64 rows x 128 B, 128-byte swizzle
 constexpr uint32_t kOffM0r = kOffMg + 8192;       // M rounded to bf16, as fp32, 16 KB
-constexpr uint32_t kOffBar = kOffM0r + 16384;
+constexpr uint32_t kOffRope = kOffM0r + 16384;    // 3D RoPE cos/sin tables, 8 KB
+constexpr uint32_t kOffBar = kOffRope + 4 * kRopeTabMaxFloats;
 enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarGather, kBarO, kBarDrain, kNumBars };
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
@@ -79,6 +80,22 @@ constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
 constexpr uint32_t kOffMst = kOffK + 32768;       // own rows of M' in bf16, <= 4 KB
 constexpr uint32_t kOffSend = kOffV;              // partial product, 64 rows x 512 B
 constexpr uint32_t kOffOut = kOffV;               // output tiles, 3 x 16 KB (after the gather)
+
+#ifdef GDN_TRACE
+// Phase timeline (globaltimer ns) of the first kTraceHeads heads, per CTA of
+// the cluster, for pipeline analysis builds only: [head][rank][event].
+constexpr int kTraceHeads = 8, kTraceEvents = 16;
+__device__ unsigned long long g_step_trace[kTraceHeads * 4 * kTraceEvents];
+#define GDN_STEP_EV(ev)                                                                          \
+  do {                                                                                           \
+    if (bh < kTraceHeads && n == 0)                                                              \
+      g_step_trace[(bh * 4 + (int)rank) * kTraceEvents + (ev)] = globaltimer_ns();               \
+  } while (0)
+#else
+#define GDN_STEP_EV(ev) \
+  do {                  \
+  } while (0)
+#endif
 
 // Status bits (shared with the scan kernel's numbering scheme, high bits).
 enum : uint32_t {
@@ -168,6 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   const int nq = (nrows + 127) / 128;   // 128-row read-out tiles
   auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * i; };
   Ctl ctl{sb + kOffAbort, p.status, p.timeout_ns, P};
+  {
+    const int n = 0;
+    if (threadIdx.x == 0) GDN_STEP_EV(10);   // kernel entry
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
@@ -199,6 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   cluster_sync();   // every CTA's barriers are initialised
+  {
+    const int n = 0;
+    if (threadIdx.x == 0) GDN_STEP_EV(11);   // past the first cluster barrier
+  }
   const uint32_t tmem = ld_shared_u32(sb + kOffTmemPtr);
   bool issued_mma = false;
   int last = -1;          // the last frame started (its barrier phases may be in flight)
@@ -206,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 
   for (int n = 0;; ++n) {
     const uint32_t ph = (uint32_t)(n & 1);   // phase parity of every per-frame barrier
+    if (threadIdx.x == 0) GDN_STEP_EV(0);
     int frame = bh;                          // index along the tensors' frame axis
     if (kStream) {
       // ------------------------------------------------------------ 0. next frame or stop
@@ -259,6 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     // swizzle only permutes whole 16-byte chunks of a row, and a chunk holds 4
     // whole pairs: physical chunk c of local row rho is logical chunk c ^ (rho & 7).
     if (p.rope && nbox > 0) {
+      // cos/sin tables of this frame and of the grid rows this CTA's tiles
+      // touch (zero-filled rows past S included), built while the tiles land
+      const int hlo = r0 / p.rp.grid_w;
+      const int nh = (r0 + nbox * kBox - 1) / p.rp.grid_w - hlo + 1;
+      const bool tab = rope_tab_floats(p.rp, nh) <= kRopeTabMaxFloats;
+      float* rtab = reinterpret_cast<float*>(smem_raw + (sb - smem_u32(smem_raw)) + kOffRope);
+      if (tab) rope_tab_build(p.rp, rtab, p.rp.t0 + n, hlo, nh);
       const bool kv_ok = warp_wait(bar(kBarKv), ph, ctl, kStLoad);
       const bool q_ok = warp_wait(bar(kBarQ), ph, ctl, kStLoad);
       if (kv_ok && q_ok) {
@@ -269,7 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
           const int rho = ce >> 3, cp = ce & 7;
           const uint32_t addr = sb + (which ? kOffQ : kOffK) + (uint32_t)rho * 128u + (uint32_t)cp * 16u;
           uint4 v = ld_shared_u4(addr);
-          rope_chunk(p.rp, p.rp.t0 + n, r0 + rho, cp ^ (rho & 7), v);
+          if (tab)
+            rope_chunk_tab(p.rp, rtab, hlo, nh, r0 + rho, cp ^ (rho & 7), v);
+          else
+            rope_chunk(p.rp, p.rp.t0 + n, r0 + rho, cp ^ (rho & 7), v);
           st_shared_v4(addr, v);
         }
         fence_proxy_async_cta();   // rotated tiles visible to the tensor cores
@@ -292,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         }
         mma_commit(bar(kBarMma));
         issued_mma = true;
+        GDN_STEP_EV(1);   // K and V landed, partial product issued
       }
     }
 
@@ -335,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         fence_proxy_async_cta();   // staged rows visible to the bulk copy
         __syncwarp();
         if (lane == 0) {
+          if (warp == 0) GDN_STEP_EV(2);   // partial product staged
           const uint32_t dst = (uint32_t)(warp * P / 4);
           const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
           bulk_copy_to_cluster(mapa(sb + kOffRed + slot_row * 512u, dst),
@@ -346,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 
     // -------------------------------------------------------------- 4. recurrence, own rows
     const bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed);
+    if (threadIdx.x == 0) GDN_STEP_EV(3);   // every partial received
     __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
     if (red_ok && !aborted(ctl)) {
       const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 K^T K (0 without delta)
@@ -419,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     fence_proxy_async_cta();   // M' rows visible to the bulk copies
     __syncthreads();
     // -------------------------------------------------------------- 5. all-gather of M' (bf16)
+    if (threadIdx.x == 0) GDN_STEP_EV(4);   // own rows of M' ready
     if (threadIdx.x == 0 && red_ok && !aborted(ctl)) {
       for (int d = 0; d < P; ++d)
         bulk_copy_to_cluster(mapa(sb + kOffMg + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
@@ -429,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (warp == 1 && lane == 0 && nq > 0) {
       if (wait_bar(bar(kBarGather), ph, ctl, kStGather) && wait_bar(bar(kBarQ), ph, ctl, kStLoad)) {
         tc_fence_after();
+        GDN_STEP_EV(5);   // gathered M' and Q present
         constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 1);   // Q K-major, M' MN-major
         for (int i = 0; i < nq; ++i) {
 #pragma unroll
@@ -477,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
           fence_proxy_async_cta();
         }
         named_bar_sync(1 + grp, 128);   // every warp of the group arrives, ok or not
+        if (qd == 0 && lane == 0 && grp == 0) GDN_STEP_EV(6);   // output tiles staged
         if (qd == 0 && lane == 0 && !aborted(ctl)) {
           const uint64_t pol = policy_evict_first();
           for (int i = grp; i < nq; i += 2) {
@@ -487,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
               tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, frame, pol);
           }
           bulk_commit();
+          if (grp == 0) GDN_STEP_EV(7);   // stores issued
           if (kStream)
             bulk_wait0();        // the frame is done only once its rows are written
           else
@@ -531,6 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   }
 
   // ---------------------------------------------------------------- exit
+  {
+    const int n = 0;
+    if (threadIdx.x == 0) GDN_STEP_EV(8);   // frame loop left
+  }
   if (kStream && p.state_out && !aborted(ctl)) {
     // this CTA's rows of the final state, fp32, kept on chip across the frames
     for (int e = threadIdx.x; e < R * kD; e += kThreads) {
@@ -567,6 +614,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  {
+    const int n = 0;
+    if (threadIdx.x == 0) GDN_STEP_EV(9);   // end
   }
 }
 
@@ -723,5 +774,12 @@ cudaError_t launch_stream_bf16(const Problem& pr, const StreamQueue& q, const Ro
   cudaLaunchConfig_t cfg = launch_config<4, true>((long long)pr.B * pr.H, pr.stream, attr);
   return cudaLaunchKernelEx(&cfg, gdn_step_kernel<4, true>, p);
 }
+
+#ifdef GDN_TRACE
+extern "C" __attribute__((visibility("default"))) int gdn_trace_step_copy(void* dst, size_t bytes) {
+  const size_t n = sizeof(g_step_trace) < bytes ? sizeof(g_step_trace) : bytes;
+  return cudaMemcpyFromSymbol(dst, g_step_trace, n) == cudaSuccess ? (int)n : -1;
+}
+#endif
 
 }  // namespace gdn

@@ -314,6 +314,7 @@ class FrameStream:
         _check(self.out, "out", torch.bfloat16, q.shape, dev)
         self.state = torch.empty((B, H, D, D), dtype=torch.float32, device=dev) if want_state else None
         self.counters = torch.zeros(2, dtype=torch.int64, pin_memory=True)   # posted, done
+        self._c = self.counters.numpy()     # the same pinned words, without torch's dispatch
         self.slots = torch.zeros(R, dtype=torch.int32, device=dev)
         self.stream = stream or torch.cuda.Stream(dev)
         self.ring, self.posted = R, 0
@@ -333,23 +334,26 @@ class FrameStream:
     def post(self, frames=1):
         """Frames posted so far += frames (their slots must hold their inputs)."""
         self.posted += frames
-        self.counters[0] = self.posted
+        self._c[0] = self.posted
 
     def done(self) -> int:
-        return int(self.counters[1])
+        return int(self._c[1])
 
     def wait(self, n, timeout_s=10.0):
         """Polls until frames 0..n-1 are done; returns the time it waited."""
         import time
+        c = self._c
+        if c[1] >= n:
+            return 0.0
         t0 = time.perf_counter()
-        while int(self.counters[1]) < n:
+        while c[1] < n:
             if time.perf_counter() - t0 > timeout_s:
-                raise TimeoutError(f"frame stream: {int(self.counters[1])} of {n} frames done")
+                raise TimeoutError(f"frame stream: {int(c[1])} of {n} frames done")
         return time.perf_counter() - t0
 
     def close(self):
         """Stops the kernel after the posted frames; returns the final state."""
-        self.counters[0] = self.posted + self.STOP
+        self._c[0] = self.posted + self.STOP
         self.stream.synchronize()
         st = device_status()
         if st != 0:
