@@ -63,6 +63,9 @@ def parse():
                     help="run only the first N frames of the workload (profiling captures)")
     ap.add_argument("--step-calls", type=int, default=961,
                     help="gdn_frame_step calls timed one by one for the step latency (0: skip)")
+    ap.add_argument("--no-stream", action="store_true",
+                    help="skip the streaming-launch latency (a persistent kernel that waits for "
+                         "host posts: never run it under a profiler's replay)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the short, stress and conv workloads (profiling captures)")
     ap.add_argument("--extra-steps", type=int, default=20,
@@ -514,7 +517,7 @@ def main():
     # The same rollout through the frame queue: one persistent launch, frames
     # posted one at a time by the host, each timed from post to done.
     stream_lat = None
-    if args.step_calls > 0:
+    if args.step_calls > 0 and not args.no_stream:
         n = min(args.step_calls, wl.T)
         ring = lambda x: x[:, :, :n].permute(2, 0, 1, *range(3, x.dim())).contiguous()
         rings = [ring(x) for x in (q, k, v, g, be)]
@@ -577,6 +580,10 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
+    clock_rec = clocks.summary()
+    if clock_rec.get("sm_mhz"):
+        # time x clock, to compare runs on boxes whose clocks differ
+        clock_rec["ms_per_step_x_sm_ghz"] = max_ms / args.steps * clock_rec["sm_mhz"] / 1e3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
@@ -591,7 +598,7 @@ def main():
         "gpu_launches": args.steps,
         "hbm_gbs": roof["achieved"],
         "roofline": roof,
-        "clocks": clocks.summary(),
+        "clocks": clock_rec,
         "e2e": e2e,
         "step_latency": step_lat,
         "stream_latency": stream_lat,

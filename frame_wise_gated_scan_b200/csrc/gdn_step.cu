@@ -190,26 +190,44 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0) GDN_STEP_EV(10);   // kernel entry
   }
 
+  // Issues the TMA loads of this CTA's rows of frame `frame` (thread 0).
+  auto issue_loads = [&](int frame) {
+    if (nbox > 0) {
+      const uint64_t pol = policy_evict_first();   // read once
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
+      for (int b = 0; b < nbox; ++b) {
+        tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
+        tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
+      }
+      mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
+      for (int b = 0; b < nbox; ++b)
+        tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, frame, pol);
+    }
+  };
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
+    if (!kStream) issue_loads(bh);   // a single frame is known now: start its loads at once
   }
   // The initial state, whole, in every CTA, with its bf16 rounding (the
-  // operand of the product A' M). It is read here, before the first cluster
-  // barrier, and the final state is written only after it: so
-  // state_in == state_out is safe.
+  // operand of the product A' M): all of a thread's loads first, then the
+  // stores. It is read here, before the first cluster barrier, and the final
+  // state is written only after it: so state_in == state_out is safe.
   {
+    constexpr int kPer = kD * kD / 4 / kThreads;   // float4 per thread
+    float4 x[kPer];
     const float4* src = reinterpret_cast<const float4*>(p.state_in + (size_t)bh * kD * kD);
-    for (int i = threadIdx.x; i < kD * kD / 4; i += kThreads) {
-      const float4 x = p.state_in ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kOffM0 + 16u * i),
-                   "f"(x.x), "f"(x.y), "f"(x.z), "f"(x.w)
-                   : "memory");
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kOffM0r + 16u * i),
-                   "f"(bf16_round(x.x)), "f"(bf16_round(x.y)), "f"(bf16_round(x.z)),
-                   "f"(bf16_round(x.w))
-                   : "memory");
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      x[i] = p.state_in ? src[threadIdx.x + i * kThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4* m0 = reinterpret_cast<float4*>(smem_raw + (sb - smem_u32(smem_raw)) + kOffM0);
+    float4* m0r = reinterpret_cast<float4*>(smem_raw + (sb - smem_u32(smem_raw)) + kOffM0r);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      m0[threadIdx.x + i * kThreads] = x[i];
+      m0r[threadIdx.x + i * kThreads] = make_float4(bf16_round(x[i].x), bf16_round(x[i].y),
+                                                    bf16_round(x[i].z), bf16_round(x[i].w));
     }
   }
   if (warp == 0) {
@@ -266,18 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0) {
       mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
       mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
-      if (nbox > 0) {
-        const uint64_t pol = policy_evict_first();   // read once
-        mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
-        for (int b = 0; b < nbox; ++b) {
-          tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
-          tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
-        }
-        mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
-        for (int b = 0; b < nbox; ++b)
-          tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, frame, pol);
-        loads_issued = true;
-      }
+      if (kStream) issue_loads(frame);   // a single frame's loads went out in the prologue
+      loads_issued = nbox > 0;
     }
 
     // -------------------------------------------------------------- 1b. 3D RoPE (optional)

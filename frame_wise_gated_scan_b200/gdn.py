@@ -115,6 +115,17 @@ def _stream_handle(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def step_args(q, k, v, gamma, beta, state_in, state_out, out, stream=None):
+    """The raw argument list of gdn_frame_step for these tensors, for callers
+    that issue many calls on the same buffers: lib().gdn_frame_step(*args)
+    then costs one ctypes call. The tensors are checked once, here."""
+    frame_step(q, k, v, gamma, beta, state_in, out=out, state_out=state_out)   # validates
+    B, H, S, D = q.shape
+    stream = stream or torch.cuda.current_stream(q.device)
+    return [_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(state_out),
+            _ptr(out), B, H, S, D, ctypes.c_void_p(stream.cuda_stream)]
+
+
 def _check(t, name, dtype, shape, device):
     if t.dtype != dtype:
         raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
@@ -184,8 +195,11 @@ def _call(step: bool, q, k, v, gamma, beta, state_in, out, state_out, want_state
         fn = L.gdn_frame_step if dt == torch.bfloat16 else L.gdn_frame_step_f32
     else:
         fn = L.gdn_frame_scan if dt == torch.bfloat16 else L.gdn_frame_scan_f32
-    with torch.cuda.device(device):
+    if device.index == torch.cuda.current_device():
         st = fn(*args)
+    else:
+        with torch.cuda.device(device):
+            st = fn(*args)
     if st != 0:
         raise GdnError(st, fn.__name__)
     return out, state_out
