@@ -376,40 +376,70 @@ class FrameStream:
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,
-                    staging=None, out_host=None, state_host=None):
+                    staging=None, out_host=None, state_host=None, groups=4):
     """End-to-end call on HOST tensors: copies the inputs to the GPU, runs the
     scan there, copies out and the final state back, and waits for them.
 
-    Pass pinned tensors for asynchronous copies. `staging` may hold reusable
-    device buffers (a dict filled on the first call) and out_host/state_host
-    reusable pinned outputs."""
+    Heads are independent and contiguous in [B,H,T,S,D], so the work is cut
+    into `groups` groups of heads and pipelined over three streams: the
+    inputs of one group cross PCIe while the previous group is scanned and the
+    one before it is copied back. Pass pinned tensors for asynchronous copies.
+    `staging` may hold reusable device buffers (a dict filled on the first
+    call) and out_host/state_host reusable pinned outputs. Returns
+    (out_host, state_host) once everything is back."""
     device = torch.device(device or "cuda")
     stream = stream or torch.cuda.current_stream(device)
     staging = {} if staging is None else staging
-    with torch.cuda.device(device), torch.cuda.stream(stream):
-        def dev(name, t):
-            if t is None:
-                return None
+    B, H, T, S, D = q.shape
+    heads = B * H
+    sshape = (B, H, D, D)
+    if out_host is None:
+        out_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if state_host is None:
+        state_host = torch.empty(sshape, dtype=torch.float32, pin_memory=True)
+    with torch.cuda.device(device):
+        def dev(name, shape, dtype):
             buf = staging.get(name)
-            if buf is None or buf.shape != t.shape or buf.dtype != t.dtype:
-                buf = torch.empty(t.shape, dtype=t.dtype, device=device)
+            if buf is None or tuple(buf.shape) != tuple(shape) or buf.dtype != dtype:
+                buf = torch.empty(shape, dtype=dtype, device=device)
                 staging[name] = buf
-            buf.copy_(t, non_blocking=True)
             return buf
-        dq, dk, dv = dev("q", q), dev("k", k), dev("v", v)
-        dg, db, ds = dev("gamma", gamma), dev("beta", beta), dev("state_in", state_in)
-        if "out" not in staging or staging["out"].shape != q.shape or staging["out"].dtype != q.dtype:
-            staging["out"] = torch.empty(q.shape, dtype=q.dtype, device=device)
-        D = q.shape[-1]
-        sshape = (q.shape[0], q.shape[1], D, D)
-        if "state_out" not in staging or tuple(staging["state_out"].shape) != sshape:
-            staging["state_out"] = torch.empty(sshape, dtype=torch.float32, device=device)
-        frame_scan(dq, dk, dv, dg, db, ds, out=staging["out"], state_out=staging["state_out"])
-        if out_host is None:
-            out_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-        if state_host is None:
-            state_host = torch.empty(sshape, dtype=torch.float32, pin_memory=True)
-        out_host.copy_(staging["out"], non_blocking=True)
-        state_host.copy_(staging["state_out"], non_blocking=True)
+        flat = lambda t, *rest: t.reshape(heads, *rest)
+        hq, hk, hv = (flat(x, 1, T, S, D) for x in (q, k, v))
+        hg, hb = flat(gamma, 1, T), flat(beta, 1, T)
+        hs = None if state_in is None else flat(state_in, 1, D, D)
+        ho, hso = flat(out_host, 1, T, S, D), flat(state_host, 1, D, D)
+        dq, dk, dv = (dev(n, (heads, 1, T, S, D), q.dtype) for n in ("q", "k", "v"))
+        dg, db = dev("gamma", (heads, 1, T), torch.float32), dev("beta", (heads, 1, T), torch.float32)
+        ds = None if state_in is None else dev("state_in", (heads, 1, D, D), torch.float32)
+        do = dev("out", (heads, 1, T, S, D), q.dtype)
+        dso = dev("state_out", (heads, 1, D, D), torch.float32)
+        copy_in = staging.setdefault("copy_in", torch.cuda.Stream(device))
+        copy_out = staging.setdefault("copy_out", torch.cuda.Stream(device))
+        n = max(1, min(int(groups), heads))
+        bounds = [heads * g // n for g in range(n + 1)]
+        copy_in.wait_stream(stream)          # the buffers are free once earlier work is done
+        copy_out.wait_stream(stream)
+        for g in range(n):
+            a, b = bounds[g], bounds[g + 1]
+            if a == b:
+                continue
+            with torch.cuda.stream(copy_in):
+                for dst, src in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (ds, hs)):
+                    if src is not None:
+                        dst[a:b].copy_(src[a:b], non_blocking=True)
+                loaded = torch.cuda.Event()
+                loaded.record(copy_in)
+            stream.wait_event(loaded)
+            with torch.cuda.stream(stream):
+                frame_scan(dq[a:b], dk[a:b], dv[a:b], dg[a:b], db[a:b],
+                           None if ds is None else ds[a:b], out=do[a:b], state_out=dso[a:b])
+                scanned = torch.cuda.Event()
+                scanned.record(stream)
+            copy_out.wait_event(scanned)
+            with torch.cuda.stream(copy_out):
+                ho[a:b].copy_(do[a:b], non_blocking=True)
+                hso[a:b].copy_(dso[a:b], non_blocking=True)
+        stream.wait_stream(copy_out)
         stream.synchronize()
     return out_host, state_host
