@@ -322,7 +322,7 @@ const char* gdn_status_string(int status) {
       return "B * H exceeds GDN_NOALLOC_MAX_HEADS (32), the fixed scratch of gdn_frame_scan_noalloc";
     case GDN_ERR_FLAGS: return "flags holds bits other than GDN_FLAG_NO_DELTA";
     case GDN_ERR_UNSUPPORTED:
-      return "sizes the call's kernel does not take (gdn_frame_step_rope: D = 64, S <= 1536; "
+      return "sizes the call's kernel does not take (gdn_frame_step_rope: D = 64, S <= 1408; "
              "gdn_frame_stream: the same, with every head's cluster resident at once)";
     default: return "unknown gdn_status";
   }

@@ -51,8 +51,8 @@ constexpr int kD = 64;
 constexpr int kThreads = 256;
 constexpr int kBox = 32;                          // rows per TMA box (loads and stores)
 constexpr uint32_t kBoxBytes = kBox * kD * 2;     // 4 KB
-constexpr int kRowsMax = 384;                     // rows of a frame per CTA
-constexpr uint32_t kRegion = kRowsMax * kD * 2;   // 48 KB: one CTA's rows of K, V or Q
+constexpr int kRowsMax = 352;                     // rows of a frame per CTA
+constexpr uint32_t kRegion = kRowsMax * kD * 2;   // 44 KB: one CTA's rows of K, V or Q
 constexpr uint32_t kTmemCols = 256;
 
 // Shared memory (from a 1 KB aligned base).
@@ -64,7 +64,8 @@ constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (
 constexpr uint32_t kOffMg = kOffRed + 32768;      // M' in bf16: 64 rows x 128 B, 128-byte swizzle
 constexpr uint32_t kOffM0r = kOffMg + 8192;       // M rounded to bf16, as fp32, 16 KB
 constexpr uint32_t kOffRope = kOffM0r + 16384;    // 3D RoPE cos/sin tables, 8 KB
-constexpr uint32_t kOffBar = kOffRope + 4 * kRopeTabMaxFloats;
+constexpr uint32_t kOffMst = kOffRope + 4 * kRopeTabMaxFloats;   // own rows of M' in bf16, <= 4 KB
+constexpr uint32_t kOffBar = kOffMst + 4096;
 enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarGather, kBarO, kBarDrain, kNumBars };
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
@@ -72,14 +73,17 @@ constexpr uint32_t kOffGo = kOffAbort + 4;         // streaming: the verdict of 
 constexpr uint32_t kBytes = kOffAbort + 16;
 constexpr uint32_t kSmemAlloc = kBytes + 1024;    // base alignment slack
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0, "swizzled regions are 1 KB aligned");
+static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0 && kOffMst % 1024 == 0,
+              "swizzled regions are 1 KB aligned");
 
 // Regions reused once the partial product has read K (K region) and V (V region):
 constexpr uint32_t kOffArow = kOffK + 16384;      // A' rows (fp32 holding bf16 values), <= 8 KB
 constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
-constexpr uint32_t kOffMst = kOffK + 32768;       // own rows of M' in bf16, <= 4 KB
+// (the own rows of M' have a region of their own: the all-gather copies read
+// them while the next frame's loads may already fill the K region)
 constexpr uint32_t kOffSend = kOffV;              // partial product, 64 rows x 512 B
-constexpr uint32_t kOffOut = kOffV;               // output tiles, 3 x 16 KB (after the gather)
+// Output tiles (after the gather): tiles 0 and 1 in the V region, tile 2 at the
+// start of the K region (free by then; its A' and c rows sit further on).
 
 #ifdef GDN_TRACE
 // Phase timeline (globaltimer ns) of the first kTraceHeads heads, per CTA of
@@ -273,8 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       break;
     }
     last = n;
-    const float g = __ldg(p.gamma + frame);
-    const float be = __ldg(p.beta + frame);
+    // plain loads: in a frame queue the host refills slots between frames
+    const float g = *reinterpret_cast<const volatile float*>(p.gamma + frame);
+    const float be = *reinterpret_cast<const volatile float*>(p.beta + frame);
 
     // -------------------------------------------------------------- 1. loads of the frame
     // The exchange barriers are armed here. A peer's data for this frame can
@@ -510,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
               for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
             }
             tmem_wait_ld();
-            const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+            const uint32_t tile = sb + (i < 2 ? kOffV + (uint32_t)i * 16384u : kOffK);
             const uint32_t row = (uint32_t)(qd * 32 + lane);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -532,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
           for (int i = grp; i < nq; i += 2) {
             const int y0 = r0 + 128 * i;
             const int y1 = min(r1, y0 + 128);
-            const uint32_t tile = sb + kOffOut + (uint32_t)i * 16384u;
+            const uint32_t tile = sb + (i < 2 ? kOffV + (uint32_t)i * 16384u : kOffK);
             for (int y = y0; y < y1; y += kBox)
               tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, frame, pol);
           }
@@ -733,6 +738,8 @@ int stream_resident_clusters() {
 }
 
 }  // namespace
+
+int step_rows_max() { return kRowsMax; }
 
 int step_ctas_per_head(int B, int H, int T, int S, int D) {
   if (D != kD || T != 1) return 0;

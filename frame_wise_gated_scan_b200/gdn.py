@@ -305,9 +305,16 @@ class FrameStream:
 
     q, k, v, out: [ring, B, H, S, D] bf16 rings and gamma, beta: [ring, B, H]
     fp32 rings on the device; frame n lives in slot n % ring. Fill a slot
-    (from pinned host memory, or before the launch), then post(); wait(n)
-    returns once frames 0..n-1 are complete. close() stops the kernel and
-    returns the final state. The counters live in pinned host memory.
+    (before the launch, or by copies from pinned host memory), then post();
+    wait(n) returns once frames 0..n-1 are complete. close() stops the kernel
+    and returns the final state. The counters live in pinned host memory.
+
+    While the launch runs it holds its SMs and waits for the host, so between
+    construction and close() the host may only post, wait, and copy between
+    pinned host memory and pre-allocated device buffers on streams of its own.
+    A kernel on the default stream, or an allocation, can be ordered after
+    the running launch by CUDA's implicit synchronisation and then wait for it
+    (the launch gives up after idle_timeout_s and reports a timeout).
     """
 
     STOP = -(1 << 63)    # bit 63 of the posted counter, as a signed int64
@@ -331,6 +338,7 @@ class FrameStream:
         self._c = self.counters.numpy()     # the same pinned words, without torch's dispatch
         self.slots = torch.zeros(R, dtype=torch.int32, device=dev)
         self.stream = stream or torch.cuda.Stream(dev)
+        self.stream.wait_stream(torch.cuda.current_stream(dev))   # the zeroed counters, the rings
         self.ring, self.posted = R, 0
         self._keep = (q, k, v, gamma, beta, state_in)
         base = self.counters.data_ptr()

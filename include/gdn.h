@@ -244,7 +244,7 @@ GDN_API int gdn_rope3d(const void* x, void* y, int B, int H, int T, int S, int D
  * any contraction reads them, so the rotated q and k never travel to HBM.
  * The result equals gdn_rope3d on q and on k followed by gdn_frame_step_ex,
  * bit for bit. Takes the sizes the row-split kernel takes (gdn_plan reports
- * GDN_KERNEL_STEP: D = 64, S <= 1536), else GDN_ERR_UNSUPPORTED; flags as in
+ * GDN_KERNEL_STEP: D = 64, S <= 1408), else GDN_ERR_UNSUPPORTED; flags as in
  * gdn_frame_step_ex. grid_w >= 1 and frame_index >= 0 (else GDN_ERR_SHAPE). */
 GDN_API int gdn_frame_step_rope(const void* q, const void* k, const void* v,
                    const float* gamma, const float* beta,
@@ -281,7 +281,10 @@ GDN_API int gdn_frame_step_rope(const void* q, const void* k, const void* v,
  * gdn_device_status() reports GDN_ERR_TIMEOUT. Only host writes to `posted`
  * (and copies by the copy engines) may feed it: work on the same GPU that the
  * caller waits for before posting could find no free SM while the kernel
- * holds them. Sizes: those of the row-split kernel (D = 64, S <= 1536) with
+ * holds them. Launch it on a non-blocking stream, and while it runs issue no
+ * work that CUDA's implicit synchronisation could order after it (work on the
+ * legacy default stream, device or pinned allocations): the caller would
+ * wait for a launch that waits for the caller, until the idle bound. Sizes: those of the row-split kernel (D = 64, S <= 1408) with
  * every head's cluster resident at once (B * H up to about 33 on a B200), else
  * GDN_ERR_UNSUPPORTED. Update and precision as gdn_frame_step; flags as in
  * gdn_frame_step_ex. Allocates nothing. */

@@ -121,6 +121,6 @@ def test_conv_rope_and_fused_step_validate_on_the_host(L):
     args = [p(0x1000000), p(0x2000000), p(0x3000000), p(0x4000000), p(0x5000000), None, None,
             p(0x6000000)]
     assert L.gdn_frame_step_rope(*args, 1, 2, 64, 128, 8, 0, 0, None) == -10          # D = 128
-    assert L.gdn_frame_step_rope(*args, 1, 2, 2000, 64, 8, 0, 0, None) == -10         # S too large
+    assert L.gdn_frame_step_rope(*args, 1, 2, 1409, 64, 8, 0, 0, None) == -10         # S too large
     assert L.gdn_frame_step_rope(*args, 1, 2, 64, 64, 0, 0, 0, None) == -2            # grid_w = 0
     assert L.gdn_frame_step_rope(*args, 1, 2, 64, 64, 8, 0, 2, None) == -9            # flags

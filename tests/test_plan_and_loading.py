@@ -36,8 +36,8 @@ def test_plan_rules_that_hold_on_any_machine(monkeypatch):
     monkeypatch.delenv("GDN_STEP_CTAS", raising=False)
     # a single frame: the row-split kernel, 4 CTAs per head share the rows
     assert gdn.plan(1, 32, 1, 880, 64) == (STEP, 4)
-    assert gdn.plan(4, 16, 1, 1536, 64) == (STEP, 4)       # 384 rows per CTA, its limit
-    assert gdn.plan(1, 32, 1, 1537, 64) == (TC, 1)         # more rows: one CTA streams them
+    assert gdn.plan(4, 16, 1, 1408, 64) == (STEP, 4)       # 352 rows per CTA, its limit
+    assert gdn.plan(1, 32, 1, 1409, 64) == (TC, 1)         # more rows: one CTA streams them
     assert gdn.plan(1, 2, 1, 1, 64) == (STEP, 4)
     assert gdn.plan(1, 2, 1, 64, 128) == (TC, 2)           # D = 128: producer + reader CTAs
     monkeypatch.setenv("GDN_STEP_CTAS", "2")
