@@ -95,9 +95,20 @@ __device__ unsigned long long g_step_trace[kTraceHeads * 4 * kTraceEvents];
     if (bh < kTraceHeads && n == 0)                                                              \
       g_step_trace[(bh * 4 + (int)rank) * kTraceEvents + (ev)] = globaltimer_ns();               \
   } while (0)
+// Streaming launch: [frame][rank][0: frame taken, 1: frame counted done], head 0.
+constexpr int kTraceFrames = 64;
+__device__ unsigned long long g_stream_trace[kTraceFrames * 4 * 2];
+#define GDN_STREAM_EV(ev)                                                              \
+  do {                                                                                 \
+    if (bh == 0 && n < kTraceFrames)                                                   \
+      g_stream_trace[(n * 4 + (int)rank) * 2 + (ev)] = globaltimer_ns();               \
+  } while (0)
 #else
 #define GDN_STEP_EV(ev) \
   do {                  \
+  } while (0)
+#define GDN_STREAM_EV(ev) \
+  do {                    \
   } while (0)
 #endif
 
@@ -194,11 +205,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0) GDN_STEP_EV(10);   // kernel entry
   }
 
+  // The initial state arrives with the first frame's K and V (single frame:
+  // one bulk copy counted on the same barrier) or is copied by the threads
+  // (streaming launch, once).
+  const bool state_bulk = !kStream && p.state_in != nullptr;
   // Issues the TMA loads of this CTA's rows of frame `frame` (thread 0).
   auto issue_loads = [&](int frame) {
+    if (state_bulk) {
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes + kD * kD * 4u);
+      bulk_load_global(sb + kOffM0, p.state_in + (size_t)bh * kD * kD, kD * kD * 4u, bar(kBarKv));
+    } else if (nbox > 0) {
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
+    }
     if (nbox > 0) {
       const uint64_t pol = policy_evict_first();   // read once
-      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
       for (int b = 0; b < nbox; ++b) {
         tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
         tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
@@ -214,25 +234,24 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     fence_mbar_init();
     if (!kStream) issue_loads(bh);   // a single frame is known now: start its loads at once
   }
-  // The initial state, whole, in every CTA, with its bf16 rounding (the
-  // operand of the product A' M): all of a thread's loads first, then the
-  // stores. It is read here, before the first cluster barrier, and the final
-  // state is written only after it: so state_in == state_out is safe.
-  {
+  // Generic pointer to the aligned shared memory, for plain loads and stores
+  // the compiler may schedule.
+  float* const smf = reinterpret_cast<float*>(smem_raw + (sb - smem_u32(smem_raw)));
+  // The initial state, whole, in every CTA. A single frame takes it by the
+  // bulk copy above, which lands before this CTA's partial product can go out,
+  // so every CTA has read it before any CTA writes the final state (after all
+  // partials are in): state_in == state_out is safe. Otherwise the threads
+  // copy it here (or write zeros), before the first cluster barrier.
+  if (!state_bulk) {
     constexpr int kPer = kD * kD / 4 / kThreads;   // float4 per thread
     float4 x[kPer];
     const float4* src = reinterpret_cast<const float4*>(p.state_in + (size_t)bh * kD * kD);
 #pragma unroll
     for (int i = 0; i < kPer; ++i)
       x[i] = p.state_in ? src[threadIdx.x + i * kThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4* m0 = reinterpret_cast<float4*>(smem_raw + (sb - smem_u32(smem_raw)) + kOffM0);
-    float4* m0r = reinterpret_cast<float4*>(smem_raw + (sb - smem_u32(smem_raw)) + kOffM0r);
+    float4* m0 = reinterpret_cast<float4*>(smf + kOffM0 / 4);
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      m0[threadIdx.x + i * kThreads] = x[i];
-      m0r[threadIdx.x + i * kThreads] = make_float4(bf16_round(x[i].x), bf16_round(x[i].y),
-                                                    bf16_round(x[i].z), bf16_round(x[i].w));
-    }
+    for (int i = 0; i < kPer; ++i) m0[threadIdx.x + i * kThreads] = x[i];
   }
   if (warp == 0) {
     tmem_alloc(sb + kOffTmemPtr, kTmemCols);
@@ -269,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
           __nanosleep(256);
         }
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + kOffGo), "r"(go) : "memory");
+        GDN_STREAM_EV(0);
       }
       __syncthreads();
       if (ld_shared_u32(sb + kOffGo) == 0 || aborted(ctl)) break;
@@ -290,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
       mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
       if (kStream) issue_loads(frame);   // a single frame's loads went out in the prologue
-      loads_issued = nbox > 0;
+      loads_issued = nbox > 0 || state_bulk;
     }
 
     // -------------------------------------------------------------- 1b. 3D RoPE (optional)
@@ -396,7 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     }
 
     // -------------------------------------------------------------- 4. recurrence, own rows
-    const bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed);
+    bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed);
+    // the bulk-copied initial state has landed (a CTA without rows has not
+    // waited on that barrier yet)
+    if (state_bulk && n == 0) red_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad) && red_ok;
     if (threadIdx.x == 0) GDN_STEP_EV(3);   // every partial received
     __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
     if (red_ok && !aborted(ctl)) {
@@ -404,15 +427,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       const float cbs = be * p.s;                    // c = beta s K^T V
       for (int e = threadIdx.x; e < R * 128; e += kThreads) {
         const int il = e >> 7, nn = e & 127;
-        const uint32_t off = (uint32_t)((((nn >> 2) ^ (il & 7)) << 4) + (nn & 3) * 4);
+        const int off = ((((nn >> 2) ^ (il & 7)) << 4) + (nn & 3) * 4) / 4;
         float sum = 0.f;
 #pragma unroll
-        for (int src = 0; src < P; ++src)
-          sum += ld_shared_f32(sb + kOffRed + (uint32_t)(src * R + il) * 512u + off);
+        for (int src = 0; src < P; ++src) sum += smf[(kOffRed / 4) + (src * R + il) * 128 + off];
         if (nn < kD)
-          st_shared_f32(sb + kOffArow + (uint32_t)(il * kD + nn) * 4u, bf16_round(coef * sum));
+          smf[kOffArow / 4 + il * kD + nn] = bf16_round(coef * sum);
         else
-          st_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + nn - kD) * 4u, cbs * sum);
+          smf[kOffCrow / 4 + il * kD + nn - kD] = cbs * sum;
+      }
+      if (n == 0) {
+        // the product's operand: the state rounded to bf16 (a streaming launch
+        // keeps it up to date between frames, step 7)
+        for (int e = threadIdx.x; e < kD * kD; e += kThreads) smf[kOffM0r / 4 + e] = bf16_round(smf[kOffM0 / 4 + e]);
       }
     }
     __syncthreads();
@@ -428,12 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 #pragma unroll
       for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
       if (p.delta != 0.f) {
-#pragma unroll 4
+        const float* arow = smf + kOffArow / 4 + il * kD;
+        const float4* m0r4 = reinterpret_cast<const float4*>(smf + kOffM0r / 4);
+#pragma unroll 8
         for (int k = 0; k < kD; ++k) {
-          const float a = ld_shared_f32(sb + kOffArow + (uint32_t)(il * kD + k) * 4u);
+          const float a = arow[k];
 #pragma unroll
           for (int c4 = 0; c4 < CPT / 4; ++c4) {
-            const float4 mk = ld_shared_f4(sb + kOffM0r + (uint32_t)(k * kD + j0 + 4 * c4) * 4u);
+            const float4 mk = m0r4[(k * kD + j0) / 4 + c4];
             acc[4 * c4 + 0] = fmaf(a, mk.x, acc[4 * c4 + 0]);
             acc[4 * c4 + 1] = fmaf(a, mk.y, acc[4 * c4 + 1]);
             acc[4 * c4 + 2] = fmaf(a, mk.z, acc[4 * c4 + 2]);
@@ -446,9 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
         const int j = j0 + c;
-        const float m0 = ld_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u);
-        m1[c] = fmaf(g, m0, acc[c]) + ld_shared_f32(sb + kOffCrow + (uint32_t)(il * kD + j) * 4u);
-        if (kStream) st_shared_f32(sb + kOffM0 + (uint32_t)(gi * kD + j) * 4u, m1[c]);   // kept on chip
+        const float m0 = smf[kOffM0 / 4 + gi * kD + j];
+        m1[c] = fmaf(g, m0, acc[c]) + smf[kOffCrow / 4 + il * kD + j];
+        if (kStream) smf[kOffM0 / 4 + gi * kD + j] = m1[c];   // kept on chip
       }
       if (!kStream && p.state_out) {
         float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)bh * kD + gi) * kD + j0);
@@ -578,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       __threadfence();
       const unsigned int total = (unsigned int)(p.heads * P);
       const unsigned int slot = (unsigned int)(n % p.ring);
+      GDN_STREAM_EV(1);
       if (atomicAdd(p.frame_done + slot, 1u) == total - 1u) {
         p.frame_done[slot] = 0u;
         __threadfence_system();
@@ -616,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       const uint32_t ph = (uint32_t)(last & 1);
       if (loads_issued) {
         drain_bar(bar(kBarKv), ph, ctl, kStDrain);
-        drain_bar(bar(kBarQ), ph, ctl, kStDrain);
+        if (nbox > 0) drain_bar(bar(kBarQ), ph, ctl, kStDrain);
       }
       drain_bar(bar(kBarRed), ph, ctl, kStDrain);
       drain_bar(bar(kBarGather), ph, ctl, kStDrain);
@@ -791,6 +821,10 @@ cudaError_t launch_stream_bf16(const Problem& pr, const StreamQueue& q, const Ro
 }
 
 #ifdef GDN_TRACE
+extern "C" __attribute__((visibility("default"))) int gdn_trace_stream_copy(void* dst, size_t bytes) {
+  const size_t n = sizeof(g_stream_trace) < bytes ? sizeof(g_stream_trace) : bytes;
+  return cudaMemcpyFromSymbol(dst, g_stream_trace, n) == cudaSuccess ? (int)n : -1;
+}
 extern "C" __attribute__((visibility("default"))) int gdn_trace_step_copy(void* dst, size_t bytes) {
   const size_t n = sizeof(g_step_trace) < bytes ? sizeof(g_step_trace) : bytes;
   return cudaMemcpyFromSymbol(dst, g_step_trace, n) == cudaSuccess ? (int)n : -1;
