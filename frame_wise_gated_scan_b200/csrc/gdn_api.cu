@@ -163,17 +163,17 @@ int gdn_frame_step_rope(const void* q, const void* k, const void* v, const float
 int gdn_frame_stream(const void* q, const void* k, const void* v, const float* gamma,
                      const float* beta, const float* state_in, float* state_out, void* out, int B,
                      int H, int S, int D, int ring, const unsigned long long* posted,
-                     unsigned long long* done, unsigned int* slot_counters,
+                     unsigned long long* done, unsigned int* queue_words,
                      unsigned long long idle_timeout_ns, unsigned int flags, void* stream) {
   const int sz = check_sizes(B, H, 1, S, D);
   if (sz != GDN_OK) return sz;
   if (ring < 1 || (long long)ring * B * H > 0x7fffffffLL) return GDN_ERR_SHAPE;
   if (flags & ~GDN_FLAG_NO_DELTA) return GDN_ERR_FLAGS;
-  if (!q || !k || !v || !gamma || !beta || !out || !posted || !done || !slot_counters)
+  if (!q || !k || !v || !gamma || !beta || !out || !posted || !done || !queue_words)
     return GDN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(gamma, 4) ||
-      !aligned(beta, 4) || !aligned(posted, 8) || !aligned(done, 8) || !aligned(slot_counters, 4))
+      !aligned(beta, 4) || !aligned(posted, 8) || !aligned(done, 8) || !aligned(queue_words, 8))
     return GDN_ERR_ALIGN;
   const size_t n = (size_t)ring * B * H * S * D * 2;
   const size_t ns = (size_t)B * H * D * D * sizeof(float);
@@ -203,7 +203,7 @@ int gdn_frame_stream(const void* q, const void* k, const void* v, const float* g
   gdn::StreamQueue qd;
   qd.posted = posted;
   qd.done = done;
-  qd.slot_counters = slot_counters;
+  qd.queue_words = queue_words;
   qd.ring = ring;
   qd.idle_timeout_ns = idle_timeout_ns;
   return gdn::launch_stream_bf16(p, qd, nullptr) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

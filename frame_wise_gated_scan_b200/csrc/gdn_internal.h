@@ -53,7 +53,7 @@ cudaError_t launch_step_bf16(const Problem& p, int ctas_per_head, const RopePara
 struct StreamQueue {
   const unsigned long long* posted;   // host-mapped, device view
   unsigned long long* done;           // host-mapped, device view
-  unsigned int* slot_counters;        // device [ring], zero
+  unsigned int* queue_words;          // device [ring + 2], zero: relay (8 bytes), then a counter per slot
   int ring;
   unsigned long long idle_timeout_ns;
 };

@@ -148,6 +148,7 @@ struct StepParams {
   // frame queue (streaming launch only)
   const unsigned long long* posted;   // host-mapped: frames posted; bit 63 set: stop after them
   unsigned long long* done;           // host-mapped: frames every head has completed
+  unsigned long long* relay;          // device: CTA 0's copy of `posted`, which every CTA polls
   unsigned int* frame_done;           // device [ring]: CTAs done with the frame in each slot (0 at start)
   int ring;                           // frame slots
   int heads;                          // B * H
@@ -276,16 +277,26 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     int frame = bh;                          // index along the tensors' frame axis
     if (kStream) {
       // ------------------------------------------------------------ 0. next frame or stop
+      // Only CTA 0 reads the host's counter (PCIe); it relays the value into
+      // device memory, which every CTA polls in L2. Many CTAs reading host
+      // memory at once would queue their reads behind each other.
       if (threadIdx.x == 0) {
         uint32_t go = 0;
         const uint64_t t0 = globaltimer_ns();
         while (true) {
-          const unsigned long long v = ld_acquire_sys_u64(p.posted);
+          unsigned long long v = ld_acquire_gpu_u64(p.relay);
+          if (blockIdx.x == 0) {
+            const unsigned long long h = ld_acquire_sys_u64(p.posted);
+            if (h != v) {
+              st_release_gpu_u64(p.relay, h);
+              v = h;
+            }
+          }
           if ((v & ~(1ull << 63)) > (unsigned long long)n) { go = 1; break; }
           if (v >> 63) break;                                   // stop after the posted frames
           if (aborted(ctl)) break;
           if (globaltimer_ns() - t0 > p.idle_ns) { raise_abort(ctl, kStIdle); break; }
-          __nanosleep(256);
+          __nanosleep(64);
         }
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + kOffGo), "r"(go) : "memory");
         GDN_STREAM_EV(0);
@@ -726,6 +737,7 @@ cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, cons
   else rope_params(&p->rp, kD, 1, 0);
   p->posted = nullptr;
   p->done = nullptr;
+  p->relay = nullptr;
   p->frame_done = nullptr;
   p->ring = 1;
   p->heads = pr.B * pr.H;
@@ -812,7 +824,8 @@ cudaError_t launch_stream_bf16(const Problem& pr, const StreamQueue& q, const Ro
   if (e != cudaSuccess) return e;
   p.posted = q.posted;
   p.done = q.done;
-  p.frame_done = q.slot_counters;
+  p.relay = reinterpret_cast<unsigned long long*>(q.queue_words);
+  p.frame_done = q.queue_words + 2;
   p.ring = q.ring;
   p.idle_ns = q.idle_timeout_ns;
   cudaLaunchAttribute attr[1];

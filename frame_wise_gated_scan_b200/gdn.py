@@ -336,9 +336,11 @@ class FrameStream:
         self.out = torch.empty_like(q) if out is None else out
         _check(self.out, "out", torch.bfloat16, q.shape, dev)
         self.state = torch.empty((B, H, D, D), dtype=torch.float32, device=dev) if want_state else None
-        self.counters = torch.zeros(2, dtype=torch.int64, pin_memory=True)   # posted, done
+        # posted at word 0, done at word 16: different 128-byte lines, since the
+        # host polls one while the device reads the other
+        self.counters = torch.zeros(32, dtype=torch.int64, pin_memory=True)
         self._c = self.counters.numpy()     # the same pinned words, without torch's dispatch
-        self.slots = torch.zeros(R, dtype=torch.int32, device=dev)
+        self.slots = torch.zeros(R + 2, dtype=torch.int32, device=dev)   # relay, then per slot
         self.stream = stream or torch.cuda.Stream(dev)
         self.stream.wait_stream(torch.cuda.current_stream(dev))   # the zeroed counters, the rings
         self.ring, self.posted = R, 0
@@ -348,7 +350,7 @@ class FrameStream:
         with torch.cuda.device(dev):
             st = L.gdn_frame_stream(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
                                     _ptr(state_in), _ptr(self.state), _ptr(self.out), B, H, S, D, R,
-                                    ctypes.c_void_p(base), ctypes.c_void_p(base + 8),
+                                    ctypes.c_void_p(base), ctypes.c_void_p(base + 128),
                                     _ptr(self.slots), int(idle_timeout_s * 1e9),
                                     0 if delta else FLAG_NO_DELTA,
                                     ctypes.c_void_p(self.stream.cuda_stream))
@@ -361,18 +363,18 @@ class FrameStream:
         self._c[0] = self.posted
 
     def done(self) -> int:
-        return int(self._c[1])
+        return int(self._c[16])
 
     def wait(self, n, timeout_s=10.0):
         """Polls until frames 0..n-1 are done; returns the time it waited."""
         import time
         c = self._c
-        if c[1] >= n:
+        if c[16] >= n:
             return 0.0
         t0 = time.perf_counter()
-        while c[1] < n:
+        while c[16] < n:
             if time.perf_counter() - t0 > timeout_s:
-                raise TimeoutError(f"frame stream: {int(c[1])} of {n} frames done")
+                raise TimeoutError(f"frame stream: {int(c[16])} of {n} frames done")
         return time.perf_counter() - t0
 
     def close(self):

@@ -268,8 +268,12 @@ GDN_API int gdn_frame_step_rope(const void* q, const void* k, const void* v,
  *           once the posted frames are done.
  *   done    written by the kernel: frames 0 .. done-1 are complete for every
  *           head (their out slots are written).
- * slot_counters: device memory, ring unsigned ints, zero at the call (the
- * kernel counts the CTAs done with each slot's frame and puts it back to zero).
+ * queue_words: device memory, ring + 2 unsigned ints, 8-byte aligned, zero at
+ * the call: the kernel's relay of `posted` (one CTA reads the host counter
+ * and copies it there for the others to poll in device memory), then a count
+ * per slot of the CTAs done with its frame (put back to zero after each frame).
+ * Keep `posted` and `done` in different 128-byte lines: the host polls one
+ * while the device reads the other.
  * The caller must fill slot n % ring before posting frame n, and must not
  * refill a slot before `done` has passed the frame it held. Frames are
  * processed in order; the state is read from state_in (NULL: zero) at the
@@ -293,7 +297,7 @@ GDN_API int gdn_frame_stream(const void* q, const void* k, const void* v,
                    const float* state_in, float* state_out, void* out,
                    int B, int H, int S, int D, int ring,
                    const unsigned long long* posted, unsigned long long* done,
-                   unsigned int* slot_counters, unsigned long long idle_timeout_ns,
+                   unsigned int* queue_words, unsigned long long idle_timeout_ns,
                    unsigned int flags, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
