@@ -457,12 +457,23 @@ def main():
         s_step.zero_()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(n)]
-        host_us = []
+        # Device time per call: a short spin kernel ahead of the first event
+        # keeps the GPU busy while the host enqueues the call, so the event
+        # pair brackets the launch and the kernel, not the host's work.
+        spin_cycles = int(80e-6 * 2.0e9)
         for t in range(n):
-            h0 = time.perf_counter()
+            torch.cuda._sleep(spin_cycles)
             evs[t][0].record(stream)
             gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
             evs[t][1].record(stream)
+            torch.cuda.synchronize(device)
+        # Host time per call: the call plus a synchronize, wall clock.
+        s_step.zero_()
+        torch.cuda.synchronize(device)
+        host_us = []
+        for t in range(n):
+            h0 = time.perf_counter()
+            gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
             torch.cuda.synchronize(device)
             host_us.append((time.perf_counter() - h0) * 1e6)
         if gdn.device_status() != 0:
@@ -509,7 +520,8 @@ def main():
                     "roofline_p50": roofline(step_bytes, pct(dev_us, 50) / 1e6),
                     "final_state_rel_diff_vs_scan": state_vs_scan,
                     "kernel": KERNEL_NAMES[step_kern], "ctas_per_head": step_ctas,
-                    "how": "device: CUDA events around each call on its stream; host: call "
+                    "how": "device: CUDA events around each call on its stream, the GPU kept "
+                           "busy by a spin kernel while the host enqueues the call; host: call "
                            "plus synchronize, wall clock; back to back: one event pair around "
                            "all calls"}
         del frames

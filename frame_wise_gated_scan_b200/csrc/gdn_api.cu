@@ -44,9 +44,7 @@ int check_sizes(int B, int H, int T, int S, int D) {
   return GDN_OK;
 }
 
-// wide: may plan the all-SM scan (it allocates its scratch, so the no-alloc
-// call does not take it).
-int choose_kernel(int B, int H, int T, int S, int D, int* ctas, bool wide = true) {
+int choose_kernel(int B, int H, int T, int S, int D, int* ctas) {
   const int f = forced_kernel();
   const int step = (f == GDN_KERNEL_SIMT) ? 0 : gdn::step_ctas_per_head(B, H, T, S, D);
   if (step > 0) {
@@ -57,11 +55,6 @@ int choose_kernel(int B, int H, int T, int S, int D, int* ctas, bool wide = true
   if (tc128 > 0) {
     *ctas = tc128;
     return GDN_KERNEL_TC;
-  }
-  const int w = (f == GDN_KERNEL_SIMT || !wide) ? 0 : gdn::wide_ctas_per_head(B, H, T, S, D);
-  if (w > 0) {
-    *ctas = w;
-    return GDN_KERNEL_TC_WIDE;
   }
   const int tc = (f == GDN_KERNEL_SIMT) ? 0 : gdn::tc_ctas_per_head(B, H, T, S, D);
   if (tc > 0) {
@@ -92,7 +85,7 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   if (state_in && state_out && state_in != state_out && overlap(state_in, ns, state_out, ns))
     return GDN_ERR_ALIAS;
   int ctas = 1;
-  const int kern = elt_bytes == 4 ? GDN_KERNEL_SIMT : choose_kernel(B, H, T, S, D, &ctas, !noalloc);
+  const int kern = elt_bytes == 4 ? GDN_KERNEL_SIMT : choose_kernel(B, H, T, S, D, &ctas);
   if (rope && kern != GDN_KERNEL_STEP) return GDN_ERR_UNSUPPORTED;
   // The fixed scratch of the no-alloc call holds the transition-operand ring,
   // which only the D = 64 tensor-core kernel with more than one CTA per head uses.
@@ -124,8 +117,6 @@ int run(const void* q, const void* k, const void* v, const float* gamma, const f
   } else {
     if (kern == GDN_KERNEL_STEP)
       err = gdn::launch_step_bf16(p, ctas, rope);   // allocates nothing
-    else if (kern == GDN_KERNEL_TC_WIDE)
-      err = gdn::launch_wide_bf16(p, ctas);
     else if (kern != GDN_KERNEL_TC)
       err = gdn::launch_simt_bf16(p);   // allocates nothing either way
     else if (D == 128)

@@ -37,13 +37,6 @@ cudaError_t launch_tc_bf16(const Problem& p, int ctas_per_head);
 // GDN_NOALLOC_MAX_HEADS; calls that overlap on the GPU race on the array.
 cudaError_t launch_tc_bf16_noalloc(const Problem& p, int ctas_per_head);
 
-// tcgen05 scan over every SM (gdn_wide.cu), bf16, D = 64, T >= 2: a
-// cooperative launch of one CTA per SM; P CTAs per head run the recurrence and
-// the read-out, every CTA produces transition operands for any head. Returns
-// P for these sizes, or 0 if it does not take them (GDN_WIDE=0 turns it off).
-int wide_ctas_per_head(int B, int H, int T, int S, int D);
-cudaError_t launch_wide_bf16(const Problem& p, int ctas_per_head);
-
 // tcgen05 kernel for D = 128 (gdn_tc128.cu): a cluster of two CTAs per head,
 // producer and reader. Returns 2 if it takes these sizes, else 0.
 int tc128_ctas_per_head(int B, int H, int T, int S, int D);

@@ -144,14 +144,15 @@ struct Layout {
   static constexpr int B_MCH_FREE = B_MCH_FULL + NM;    // [NM] read-out MMAs of M_t done
   static constexpr int B_O_FULL = B_MCH_FREE + NM;
   static constexpr int B_O_FREE = B_O_FULL + 2;
-  static constexpr int B_DRAIN = B_O_FREE + 2;         // [3] one per MMA issuer
-  static constexpr int B_E1_STAGED = B_DRAIN + 3;       // [4] frame's A'/c written (4 warps)
+  static constexpr int B_DRAIN = B_O_FREE + 2;         // [7] one per MMA-issuing thread
+  static constexpr int B_E1_STAGED = B_DRAIN + 7;       // [4] frame's A'/c written (4 warps)
   static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
   static constexpr int B_STAGE = B_PUB_DONE + 4;        // [2] output tile staged (4 warps)
   static constexpr int B_CLAIM = B_STAGE + 2;           // [NCLAIM] frame of job j known
   static constexpr int NBAR = B_CLAIM + NCLAIM;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
+  static constexpr uint32_t OFF_CHAIN_CTR = OFF_ABORT + 4;    // u32: recurrence warps done with a frame
   static constexpr uint32_t OFF_CLAIM_CTR = OFF_ABORT + 16;   // u32; rank 0's counts the head's claims
   static constexpr uint32_t OFF_CLAIMS = OFF_CLAIM_CTR + 16;  // [NCLAIM] s32: frame of job j, -1 = done
   static constexpr uint32_t BYTES = OFF_CLAIMS + 4 * NCLAIM;
@@ -206,6 +207,7 @@ struct TcParams {
   float s;     // key scale 1/sqrt(D*S)
   float s2;    // its square
   float delta; // 1: delta rule; 0: GDN_FLAG_NO_DELTA, so A' = 0 and M' = gamma M + c
+  int self_issue;   // 1: the last recurrence warp issues the next frame's MMAs; 0: warp 2 does
 };
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
@@ -345,6 +347,29 @@ __device__ __forceinline__ bool wait_global_ge(const unsigned long long* ptr,
   }
 }
 
+// A'_t M_{t-1} into the recurrence accumulator, committed to `done`: A'_t
+// K-major in `ac`, M_{t-1} as two MN-major 32-column blocks from `mprev`. Both
+// in bf16: the product is small next to the exact fp32 gamma M term it is added
+// to, so its relative rounding error enters the state scaled down by |A'| / gamma.
+template <int P>
+__device__ __forceinline__ void chain_mma(uint32_t tmem, uint32_t ac, uint32_t mprev, uint32_t done) {
+  using L = Layout<P>;
+  constexpr uint32_t id_chain = idesc_bf16(64, 32, 0, 1);    // A' K-major, M half MN-major
+  tc_fence_after();
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
+      const uint32_t mb = mprev + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
+      const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
+      mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
+    }
+  }
+  mma_commit(done);
+}
+
 template <int P>
 __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<P>;
@@ -414,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mbar_init(bar(L::B_STAGE + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
-    for (int i = 0; i < 3; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
+    for (int i = 0; i < 7; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::OFF_CHAIN_CTR), "r"(0u) : "memory");
     for (int i = 0; i < L::NCLAIM; ++i) mbar_init(bar(L::B_CLAIM + i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::OFF_CLAIM_CTR), "r"(0u) : "memory");
@@ -548,32 +574,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
       drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
-  } else if (warp == 2 && lane == 0) {
+  } else if (warp == 2 && lane == 0 && !p.self_issue) {
     // ------------------------------------------------ recurrence MMA issuer
     // tcgen05.commit tracks the MMAs of the issuing thread, so each of the three
     // MMA streams has its own issuer and waits only on its own inputs.
-    constexpr uint32_t id_chain = idesc_bf16(64, 32, 0, 1);    // A' K-major, M half MN-major
     for (int t = 0; t < T; ++t) {
       if (!poll_bar(bar(L::B_M_READY), t & 1, ctl, kStMma) ||
           !poll_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma))
         break;
-      tc_fence_after();
-      const uint32_t ac = ac_slot(t % NAC);
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const uint32_t dt = tmem + L::T_CHAIN + ((uint32_t)hf << 20);   // lane offset 16
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          // A' M_{t-1} with both in bf16: the product is small next to the
-          // exact fp32 gamma M term it is added to, so its relative rounding
-          // error enters the state scaled down by |A'| / gamma.
-          const uint64_t aH = smem_desc(ac + kk * 32, 16, 1024, 2);
-          const uint32_t mb = mch((t + L::NM - 1) % L::NM) + hf * L::MB_BLOCK + kk * 2 * L::MB_SBO;
-          const uint64_t bH = smem_desc(mb, L::MB_BLOCK, L::MB_SBO, 4);
-          mma_bf16(dt, aH, bH, id_chain, kk > 0 ? 1u : 0u);
-        }
-      }
-      mma_commit(bar(L::B_CHAIN_DONE));
+      chain_mma<P>(tmem, ac_slot(t % NAC), mch((t + L::NM - 1) % L::NM), bar(L::B_CHAIN_DONE));
       GDN_TRACE_EV(0, t);
 #ifdef GDN_TRACE
       if (rank == 0 && bh < kTraceHeads && t < kTraceFrames)
@@ -690,15 +699,38 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       for (int c = 0; c < 4; ++c)
         st_shared_v4(buf + hf * L::MB_BLOCK + swz_off(row, c, L::MB_RW, 2), pack8(&m[8 * c]));
     };
+    // This warp is done with frame t - 1 (its rows of M_{t-1} written and
+    // fenced, its accumulator reads complete). Without self_issue it tells the
+    // issuer (warp 2); with it, the last of the four warps to get here issues
+    // frame t's MMAs itself, one hand-off fewer on the serial path.
+    bool issued = false;
+    auto frame_done = [&](int t) -> bool {
+      uint32_t ok = 1;
+      if (lane == 0) {
+        if (!p.self_issue) {
+          mbar_arrive(bar(L::B_M_READY));
+        } else {
+          const uint32_t old = atom_add_acq_rel_shared(sb + L::OFF_CHAIN_CTR, 1u);
+          if ((old & 3u) == 3u && t < T) {
+            ok = wait_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma) ? 1u : 0u;
+            if (ok) {
+              chain_mma<P>(tmem, ac_slot(t % NAC), mch((t + L::NM - 1) % L::NM), bar(L::B_CHAIN_DONE));
+              issued = true;
+              GDN_TRACE_EV(0, t);
+            }
+          }
+        }
+      }
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
     store_state(mch(L::NM - 1));               // M_{-1} = M_0, read by the first MMA
     fence_proxy_async_cta();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::B_M_READY));
+    bool ok = frame_done(0);
     const float* gam = p.gamma + (size_t)bh * T;
     float g_next = __ldg(gam);
-    bool ok = true;
     int t = 0;
-    for (; t < T; ++t) {
+    for (; t < T && ok; ++t) {
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
@@ -741,11 +773,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
         mbar_arrive(bar(L::B_AC_EMPTY + s));   // A'_t read by its MMA, c_t read here: slot free
         mbar_arrive(bar(L::B_MCH_FULL + t % L::NM));   // M_t ready for the read-out
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
+      ok = frame_done(t + 1);                  // next MMA operand ready; accumulator free
+    }
+    if (lane == 0 && issued) {
+      // MMAs this thread issued may still run if the loop stopped early.
+      mma_commit(bar(L::B_DRAIN + 3 + qd));
+      drain_bar(bar(L::B_DRAIN + 3 + qd), 0, ctl);
     }
     if (ok && p.state_out && rank == 0) {      // every CTA holds the same state
 #pragma unroll
@@ -988,36 +1025,23 @@ cudaError_t prepare() {
   return e;
 }
 
-// Clusters of P CTAs that can be resident at once on the current device, or
-// -1 if there is no usable device (host-only planning). Cached per device.
+// Clusters of P CTAs (one CTA per SM) that fit on the current device at
+// once, or -1 if there is no usable device (host-only planning). A cluster
+// sits inside one GPC, so clusters of 4 leave a few SMs of each GPC unused:
+// 33 fit on a 148-SM B200, about 9/40 of the SM count; clusters of 2 fill the
+// device. Only the cluster size depends on this count (the clusters never
+// wait on each other), so it comes from the SM count rather than from the
+// driver's cluster-occupancy query: that query, made before the caller's
+// large allocations, was followed by scans running 20-45 % slower.
 template <int P>
 int resident_clusters() {
-  static std::atomic<int> cache[64];            // 0: not yet known; else the count + 2
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     return -1;
   }
-  const int known = cache[dev].load(std::memory_order_acquire);
-  if (known != 0) return known - 2;
-  int n = -1;
-  if (prepare<P>() == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = P;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(P * 64, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Layout<P>::SMEM_ALLOC;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, gdn_tc_kernel<P>, &cfg) != cudaSuccess) n = -1;
-  }
-  cudaGetLastError();
-  cache[dev].store(n + 2, std::memory_order_release);
-  return n;
+  return P == 4 ? sms * 9 / 40 : sms / P;
 }
 
 // Address of g_noalloc_scratch on the current device. cudaGetSymbolAddress
@@ -1070,6 +1094,8 @@ cudaError_t launch_p(const Problem& pr, uint8_t* fixed_scratch) {
   const double sd = 1.0 / ((double)kD * (double)pr.S);
   p.s2 = (float)sd;
   p.delta = pr.delta ? 1.f : 0.f;
+  p.self_issue = 0;
+  if (const char* e = getenv("GDN_TC_SELF")) p.self_issue = atoi(e) != 0;
 
   // Ring of transition operands shared by the CTAs of each head (P > 1):
   // stream-ordered scratch, released right after the launch on the same stream.
@@ -1137,8 +1163,8 @@ int tc_ctas_per_head(int B, int H, int T, int S, int D) {
   // Largest cluster size whose clusters all fit on the device at once.
   const int c4 = resident_clusters<4>();
   const int c2 = resident_clusters<2>();
-  const int sms = 148;
-  const long long fit4 = c4 >= 0 ? c4 : sms / 4;
+  const int sms = 148;                     // planning without a device: a B200
+  const long long fit4 = c4 >= 0 ? c4 : sms * 9 / 40;
   const long long fit2 = c2 >= 0 ? c2 : sms / 2;
   if (heads <= fit4) return 4;
   if (heads <= fit2) return 2;

@@ -21,7 +21,6 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
 KERNEL_SIMT = 1
 KERNEL_TC = 2
 KERNEL_STEP = 3
-KERNEL_TC_WIDE = 4
 FLAG_NO_DELTA = 1     # GDN_FLAG_NO_DELTA: R = V, the decayed cumulative (block KV cache) form
 
 _lib = None

@@ -308,10 +308,6 @@ GDN_API int gdn_frame_stream(const void* q, const void* k, const void* v,
 #define GDN_KERNEL_TC 2     /* tcgen05 kernel, a cluster of CTAs per head */
 #define GDN_KERNEL_STEP 3   /* single-frame tcgen05 kernel (T = 1, D = 64): a cluster of
                                CTAs per head splits the frame's rows */
-#define GDN_KERNEL_TC_WIDE 4 /* tcgen05 scan over every SM (D = 64, T >= 2, B * H up to
-                               the SM count): ctas_per_head CTAs per head run the
-                               recurrence and the read-out, every CTA produces the
-                               transition operands of any head */
 GDN_API int gdn_plan(int B, int H, int T, int S, int D, int* kernel, int* ctas_per_head);
 
 /* Synchronizes the current device, then returns GDN_ERR_TIMEOUT if any kernel

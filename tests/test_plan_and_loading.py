@@ -20,13 +20,13 @@ def _built():
 
 
 @pytest.mark.skipif(torch.cuda.is_available(),
-                    reason="with a device the thresholds come from its cluster occupancy")
+                    reason="with a device the thresholds come from its SM count")
 def test_plan_without_a_device(monkeypatch):
     monkeypatch.delenv("GDN_TC_CTAS", raising=False)
-    # 148 SMs assumed: 37 clusters of 4, 74 of 2 fit at once
+    # 148 SMs assumed: 33 clusters of 4 (whole GPCs), 74 of 2 fit at once
     assert gdn.plan(1, 32, 961, 880, 64) == (TC, 4)
-    assert gdn.plan(1, 37, 2, 64, 64) == (TC, 4)
-    assert gdn.plan(1, 38, 2, 64, 64) == (TC, 2)
+    assert gdn.plan(1, 33, 2, 64, 64) == (TC, 4)
+    assert gdn.plan(1, 34, 2, 64, 64) == (TC, 2)
     assert gdn.plan(2, 37, 2, 64, 64) == (TC, 2)
     assert gdn.plan(1, 75, 2, 64, 64) == (TC, 1)
 
