@@ -144,15 +144,14 @@ struct Layout {
   static constexpr int B_MCH_FREE = B_MCH_FULL + NM;    // [NM] read-out MMAs of M_t done
   static constexpr int B_O_FULL = B_MCH_FREE + NM;
   static constexpr int B_O_FREE = B_O_FULL + 2;
-  static constexpr int B_DRAIN = B_O_FREE + 2;         // [7] one per MMA-issuing thread
-  static constexpr int B_E1_STAGED = B_DRAIN + 7;       // [4] frame's A'/c written (4 warps)
+  static constexpr int B_DRAIN = B_O_FREE + 2;         // [3] one per MMA issuer
+  static constexpr int B_E1_STAGED = B_DRAIN + 3;       // [4] frame's A'/c written (4 warps)
   static constexpr int B_PUB_DONE = B_E1_STAGED + 4;    // [4] frame published to the ring
   static constexpr int B_STAGE = B_PUB_DONE + 4;        // [2] output tile staged (4 warps)
   static constexpr int B_CLAIM = B_STAGE + 2;           // [NCLAIM] frame of job j known
   static constexpr int NBAR = B_CLAIM + NCLAIM;
   static constexpr uint32_t OFF_TMEM_PTR = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
-  static constexpr uint32_t OFF_CHAIN_CTR = OFF_ABORT + 4;    // u32: recurrence warps done with a frame
   static constexpr uint32_t OFF_CLAIM_CTR = OFF_ABORT + 16;   // u32; rank 0's counts the head's claims
   static constexpr uint32_t OFF_CLAIMS = OFF_CLAIM_CTR + 16;  // [NCLAIM] s32: frame of job j, -1 = done
   static constexpr uint32_t BYTES = OFF_CLAIMS + 4 * NCLAIM;
@@ -207,7 +206,6 @@ struct TcParams {
   float s;     // key scale 1/sqrt(D*S)
   float s2;    // its square
   float delta; // 1: delta rule; 0: GDN_FLAG_NO_DELTA, so A' = 0 and M' = gamma M + c
-  int self_issue;   // 1: the last recurrence warp issues the next frame's MMAs; 0: warp 2 does
 };
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
@@ -439,8 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     mbar_init(bar(L::B_STAGE + 1), 4);
     mbar_init(bar(L::B_CHAIN_DONE), 1);
     mbar_init(bar(L::B_M_READY), 4);
-    for (int i = 0; i < 7; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::OFF_CHAIN_CTR), "r"(0u) : "memory");
+    for (int i = 0; i < 3; ++i) mbar_init(bar(L::B_DRAIN + i), 1);
     for (int i = 0; i < L::NCLAIM; ++i) mbar_init(bar(L::B_CLAIM + i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::OFF_CLAIM_CTR), "r"(0u) : "memory");
@@ -574,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
     for (int k = it - 1; k >= 0 && k >= it - L::NQ; --k)
       drain_bar(bar(L::B_Q_FULL + k % L::NQ), (k / L::NQ) & 1, ctl);
-  } else if (warp == 2 && lane == 0 && !p.self_issue) {
+  } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------ recurrence MMA issuer
     // tcgen05.commit tracks the MMAs of the issuing thread, so each of the three
     // MMA streams has its own issuer and waits only on its own inputs.
@@ -699,38 +696,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       for (int c = 0; c < 4; ++c)
         st_shared_v4(buf + hf * L::MB_BLOCK + swz_off(row, c, L::MB_RW, 2), pack8(&m[8 * c]));
     };
-    // This warp is done with frame t - 1 (its rows of M_{t-1} written and
-    // fenced, its accumulator reads complete). Without self_issue it tells the
-    // issuer (warp 2); with it, the last of the four warps to get here issues
-    // frame t's MMAs itself, one hand-off fewer on the serial path.
-    bool issued = false;
-    auto frame_done = [&](int t) -> bool {
-      uint32_t ok = 1;
-      if (lane == 0) {
-        if (!p.self_issue) {
-          mbar_arrive(bar(L::B_M_READY));
-        } else {
-          const uint32_t old = atom_add_acq_rel_shared(sb + L::OFF_CHAIN_CTR, 1u);
-          if ((old & 3u) == 3u && t < T) {
-            ok = wait_bar(bar(L::B_AC_FULL + t % NAC), (t / NAC) & 1, ctl, kStMma) ? 1u : 0u;
-            if (ok) {
-              chain_mma<P>(tmem, ac_slot(t % NAC), mch((t + L::NM - 1) % L::NM), bar(L::B_CHAIN_DONE));
-              issued = true;
-              GDN_TRACE_EV(0, t);
-            }
-          }
-        }
-      }
-      return __shfl_sync(0xffffffffu, ok, 0) != 0;
-    };
     store_state(mch(L::NM - 1));               // M_{-1} = M_0, read by the first MMA
     fence_proxy_async_cta();
     __syncwarp();
-    bool ok = frame_done(0);
+    if (lane == 0) mbar_arrive(bar(L::B_M_READY));
     const float* gam = p.gamma + (size_t)bh * T;
     float g_next = __ldg(gam);
+    bool ok = true;
     int t = 0;
-    for (; t < T && ok; ++t) {
+    for (; t < T; ++t) {
       const float g = g_next;
       if (t + 1 < T) g_next = __ldg(gam + t + 1);
       const int s = t % NAC;
@@ -773,16 +747,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
       fence_proxy_async_cta();
       __syncwarp();
       if (lane == 0) {
+        mbar_arrive(bar(L::B_M_READY));        // next MMA operand ready; accumulator free
         mbar_arrive(bar(L::B_AC_EMPTY + s));   // A'_t read by its MMA, c_t read here: slot free
         mbar_arrive(bar(L::B_MCH_FULL + t % L::NM));   // M_t ready for the read-out
         if (warp == 4) GDN_TRACE_EV(2, t);
       }
-      ok = frame_done(t + 1);                  // next MMA operand ready; accumulator free
-    }
-    if (lane == 0 && issued) {
-      // MMAs this thread issued may still run if the loop stopped early.
-      mma_commit(bar(L::B_DRAIN + 3 + qd));
-      drain_bar(bar(L::B_DRAIN + 3 + qd), 0, ctl);
     }
     if (ok && p.state_out && rank == 0) {      // every CTA holds the same state
 #pragma unroll
@@ -1094,8 +1063,6 @@ cudaError_t launch_p(const Problem& pr, uint8_t* fixed_scratch) {
   const double sd = 1.0 / ((double)kD * (double)pr.S);
   p.s2 = (float)sd;
   p.delta = pr.delta ? 1.f : 0.f;
-  p.self_issue = 0;
-  if (const char* e = getenv("GDN_TC_SELF")) p.self_issue = atoi(e) != 0;
 
   // Ring of transition operands shared by the CTAs of each head (P > 1):
   // stream-ordered scratch, released right after the launch on the same stream.

@@ -114,15 +114,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned 
   return v;
 }
 
-// Shared-memory counter of the CTA: returns the old value; orders this
-// thread's earlier accesses before, and later ones after, the update.
-__device__ __forceinline__ uint32_t atom_add_acq_rel_shared(uint32_t addr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v)
-               : "memory");
-  return old;
-}
-
 // Non-blocking: has the phase with this parity completed? (acquire, CTA scope)
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
