@@ -114,14 +114,23 @@ def _strip_comments(src: str) -> str:
     return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
 
 
-def kernel_source_hash() -> str:
-    """SHA-256 of the kernel sources' code (comments removed)."""
+# Sources each timed scan kernel is built from (its own file, the PTX wrappers,
+# the shared waits, the internal interface and the host helpers).
+KERNEL_SOURCES = {
+    "rollout": ("gdn_tc.cu", "sm100_ptx.h", "gdn_internal.h", "gdn_host.cu"),
+    "short": ("gdn_tc.cu", "sm100_ptx.h", "gdn_internal.h", "gdn_host.cu"),
+    "stress": ("gdn_tc128.cu", "sm100_ptx.h", "gdn_wait.cuh", "gdn_internal.h", "gdn_host.cu"),
+}
+
+
+def kernel_source_hash(workload: str) -> str:
+    """SHA-256 of the code (comments removed) of the sources the workload's
+    kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "frame_wise_gated_scan_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".h")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
+    for name in sorted(KERNEL_SOURCES.get(workload, ())):
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
     return h.hexdigest()
 
 
@@ -133,7 +142,7 @@ def recorded_traffic(workload: str):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("source_sha256") != kernel_source_hash():
+    if workload not in KERNEL_SOURCES or rec.get("source_sha256") != kernel_source_hash(workload):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -426,11 +426,22 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       }
     }
 
+    // The first frame's product takes the state rounded to bf16 (a streaming
+    // launch keeps it up to date between frames, step 7). Warps 4-7 round it
+    // while warps 0-3 stage the partials, once the bulk-copied state has landed.
+    bool m0r_ok = true;
+    if (n == 0 && warp >= 4) {
+      if (state_bulk) m0r_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad);
+      if (m0r_ok && !aborted(ctl))
+        for (int e = threadIdx.x - 128; e < kD * kD; e += kThreads - 128)
+          smf[kOffM0r / 4 + e] = bf16_round(smf[kOffM0 / 4 + e]);
+    }
+
     // -------------------------------------------------------------- 4. recurrence, own rows
-    bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed);
+    bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed) && m0r_ok;
     // the bulk-copied initial state has landed (a CTA without rows has not
     // waited on that barrier yet)
-    if (state_bulk && n == 0) red_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad) && red_ok;
+    if (state_bulk && n == 0 && warp < 4) red_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad) && red_ok;
     if (threadIdx.x == 0) GDN_STEP_EV(3);   // every partial received
     __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
     if (red_ok && !aborted(ctl)) {
@@ -446,11 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
           smf[kOffArow / 4 + il * kD + nn] = bf16_round(coef * sum);
         else
           smf[kOffCrow / 4 + il * kD + nn - kD] = cbs * sum;
-      }
-      if (n == 0) {
-        // the product's operand: the state rounded to bf16 (a streaming launch
-        // keeps it up to date between frames, step 7)
-        for (int e = threadIdx.x; e < kD * kD; e += kThreads) smf[kOffM0r / 4 + e] = bf16_round(smf[kOffM0 / 4 + e]);
       }
     }
     __syncthreads();
