@@ -14,7 +14,8 @@
 // with no contraction, so it runs on CUDA cores with 16-byte accesses. Thread
 // (column, segment) owns 8 channels of one token (one 16-byte vector per
 // frame) over a run of frames, keeps the previous, current and next frame in
-// registers, and keeps eight frames of loads in flight. Warps read and write
+// registers, and keeps eight frames of loads in flight (a slot is reloaded as
+// soon as its frame is used). Warps read and write
 // 512 contiguous bytes per frame. Segments split long runs of frames across
 // threads so that small S * C still fills the GPU; a segment reads the frame
 // before it (or the cache) once.
@@ -103,14 +104,20 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_tconv_kernel(
 #pragma unroll
       for (int e = 0; e < 8; ++e) prev[e] = 0.f;
     }
-    uint4 cur = ld_stream(xc + (size_t)t0 * fs, pol);
+    // Frame f is loaded when this segment needs it: f < t1 (written here) or
+    // f == t1 (the next frame of the segment's last one), and f < T.
+    auto load = [&](int f) -> uint4 {
+      return (f < T && f <= t1) ? ld_stream(xc + (size_t)f * fs, pol) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    // Rolling prefetch: on entry to each round, cur is frame t and ahead[u]
+    // frame t+1+u. A slot is refilled, kAhead frames further on, as soon as
+    // its frame is used, so about kAhead loads stay in flight.
+    uint4 cur = load(t0);
+    uint4 ahead[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) ahead[u] = load(t0 + 1 + u);
     uint4 last = cur;
     for (int t = t0; t < t1; t += kAhead) {
-      uint4 ahead[kAhead];   // frames t+1 .. t+kAhead, loaded together
-#pragma unroll
-      for (int u = 0; u < kAhead; ++u)
-        ahead[u] = (t + 1 + u < T && t + u < t1) ? ld_stream(xc + (size_t)(t + 1 + u) * fs, pol)
-                                                 : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int u = 0; u < kAhead; ++u) {
         const int tt = t + u;
@@ -120,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_tconv_kernel(
           float xc_[8], xn[8];
           unpack8(raw, xc_);
           unpack8(ahead[u], xn);
+          if (u > 0) ahead[u - 1] = load(tt + kAhead);   // frame t + kAhead + u
           float o[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -134,7 +142,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_tconv_kernel(
           last = raw;
         }
       }
-      cur = ahead[kAhead - 1];
+      cur = ahead[kAhead - 1];                           // frame t + kAhead
+      ahead[kAhead - 1] = load(t + 2 * kAhead);          // frame t + kAhead + 1 + (kAhead - 1)
     }
     // The first segment hands the cache on: it is the thread that read
     // cache_in, so cache_in == cache_out is safe.

@@ -1,7 +1,7 @@
 // Standalone 3D RoPE of a [B][H][T][S][D] bf16 array of queries or keys (the
 // rotation and its layout are described in gdn_rope.cuh). HBM-bound: each
-// thread reads one 16-byte chunk (4 pairs) of a token row and writes it back
-// rotated; consecutive threads take consecutive chunks.
+// thread reads 16-byte chunks (4 pairs) of token rows, four at a time, and
+// writes them back rotated; consecutive threads take consecutive chunks.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -13,6 +13,7 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kBatch = 4;   // 16-byte chunks per thread and step
 
 // One block per frame: cos/sin tables of the frame first (shared memory),
 // then the frame's rows, one 16-byte chunk per thread and step. Frames whose
@@ -29,18 +30,31 @@ __global__ void __launch_bounds__(kThreads) gdn_rope_kernel(const uint4* x, uint
     if (use_tab) rope_tab_build(rp, tab, t, 0, nh);
     const uint4* xs = x + f * chunks;
     uint4* ys = y + f * chunks;
-    for (long long idx = threadIdx.x; idx < chunks; idx += kThreads) {
-      const int chunk = (int)(idx % D8);
-      const int r = (int)(idx / D8);
-      uint4 v;
-      asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "l"(xs + idx));
-      if (use_tab)
-        rope_chunk_tab(rp, tab, 0, nh, r, chunk, v);
-      else
-        rope_chunk(rp, t, r, chunk, v);
-      ys[idx] = v;
+    // kBatch chunks per thread and step, their loads issued together so that
+    // several are in flight; consecutive threads keep consecutive chunks.
+    for (long long base = threadIdx.x; base < chunks; base += kBatch * kThreads) {
+      uint4 v[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const long long idx = base + (long long)k * kThreads;
+        if (idx < chunks)
+          asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v[k].x), "=r"(v[k].y), "=r"(v[k].z), "=r"(v[k].w)
+                       : "l"(xs + idx));
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const long long idx = base + (long long)k * kThreads;
+        if (idx < chunks) {
+          const int chunk = (int)(idx % D8);
+          const int r = (int)(idx / D8);
+          if (use_tab)
+            rope_chunk_tab(rp, tab, 0, nh, r, chunk, v[k]);
+          else
+            rope_chunk(rp, t, r, chunk, v[k]);
+          ys[idx] = v[k];
+        }
+      }
     }
     __syncthreads();   // the next frame's table may replace this one
   }
