@@ -518,21 +518,45 @@ def main():
         torch.cuda.synchronize(device)
         graph_us = e0.elapsed_time(e1) * 1e3 / n
         del graph
+        # Per-step device time inside a replayed graph: event records captured
+        # between the steps (no host work, no configuration switch between
+        # consecutive kernels).
+        graph_steps = None
+        try:
+            gev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                gev[0].record()
+                for t in range(n):
+                    gdn.frame_step(*frames[t], s_step, out=o_step, state_out=s_step)
+                    gev[t + 1].record()
+            for _ in range(2):
+                s_step.zero_()
+                graph.replay()
+                torch.cuda.synchronize(device)
+            graph_steps = sorted(gev[t].elapsed_time(gev[t + 1]) * 1e3 for t in range(n))
+            del graph
+        except RuntimeError:
+            graph_steps = None
         step_bytes = inputs.algorithmic_bytes(wl, 1) + wl.heads * wl.D * wl.D * 4
         step_lat = {"calls": n, "unit": "us",
                     "device_p50": pct(dev_us, 50), "device_p99": pct(dev_us, 99),
                     "host_p50": pct(host_us, 50), "host_p99": pct(host_us, 99),
                     "back_to_back_us_per_call": b2b_us,
                     "graph_us_per_step": graph_us,
+                    "graph_step_p50": pct(graph_steps, 50) if graph_steps else None,
+                    "graph_step_p99": pct(graph_steps, 99) if graph_steps else None,
                     # q, k, v read, out written, gates, the state read and written
                     "bytes_per_call": step_bytes,
-                    "roofline_p50": roofline(step_bytes, pct(dev_us, 50) / 1e6),
+                    "roofline_p50": roofline(
+                        step_bytes, (pct(graph_steps, 50) if graph_steps else pct(dev_us, 50)) / 1e6),
                     "final_state_rel_diff_vs_scan": state_vs_scan,
                     "kernel": KERNEL_NAMES[step_kern], "ctas_per_head": step_ctas,
                     "how": "device: CUDA events around each call on its stream, the GPU kept "
-                           "busy by a spin kernel while the host enqueues the call; host: call "
-                           "plus synchronize, wall clock; back to back: one event pair around "
-                           "all calls"}
+                           "busy by a spin kernel while the host enqueues the call; graph_step: "
+                           "events between consecutive steps inside a replayed CUDA graph "
+                           "(roofline_p50 uses its p50); host: call plus synchronize, wall "
+                           "clock; back to back: one event pair around all calls"}
         del frames
 
     # The same rollout through the frame queue: one persistent launch, frames
