@@ -523,7 +523,8 @@ def main():
         # consecutive kernels).
         graph_steps = None
         try:
-            gev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            # external: captured as event record nodes of the graph
+            gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)]
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 gev[0].record()
