@@ -659,7 +659,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     // Every frame, this CTA's own included, arrives through the ring, in frame
     // order, so each slot wait below is for the next phase of its barrier. The
     // bulk load completes the slot's "full" barrier itself.
-    const uint64_t ring_pol = policy_evict_last();     // the ring (16 frames per head) stays in L2
+    // The ring keeps the normal eviction priority: the streams around it are
+    // evict-first, so it stays in L2 anyway. With evict-last, lines of rings that
+    // earlier launches left at other addresses kept their priority and crowded
+    // out the live ring: the same launch then ran up to 7x slower.
+    const uint64_t ring_pol = policy_evict_normal();
     int t = 0;
     for (; t < T; ++t) {
       const int s = t % NAC;
@@ -855,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane == 0 && warp == 8) GDN_TRACE_EV(7, j);
         uint8_t* img = p.ring + rs * L::AC_BYTES;
-        const uint64_t ring_pol = policy_evict_last();
+        const uint64_t ring_pol = policy_evict_normal();
         if (lrow < kD) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
