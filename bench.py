@@ -67,11 +67,11 @@ def parse():
                     help="skip the streaming-launch latency (a persistent kernel that waits for "
                          "host posts: never run it under a profiler's replay)")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the short, stress and conv workloads (profiling captures)")
+                    help="skip the tiny, short, stress, conv and RoPE workloads (profiling captures)")
     ap.add_argument("--extra-steps", type=int, default=20,
                     help="timed launches of each extra workload")
-    ap.add_argument("--extras", default="short,stress,conv,rope",
-                    help="comma-separated extra workloads (short, stress, conv, rope)")
+    ap.add_argument("--extras", default="tiny,short,stress,conv,rope",
+                    help="comma-separated extra workloads (tiny, short, stress, conv, rope)")
     ap.add_argument("--extra-frames", type=int, default=0,
                     help="cut the extra workloads to this many frames (profiling captures)")
     return ap.parse_args()
@@ -596,7 +596,8 @@ def main():
     if not args.no_extras and rank == 0:
         want = [x.strip() for x in args.extras.split(",") if x.strip()]
         ef = args.extra_frames
-        run = {"short": lambda: scan_workload("short", device, stream, args.extra_steps * 10, ef),
+        run = {"tiny": lambda: scan_workload("tiny", device, stream, args.extra_steps * 10, ef),
+               "short": lambda: scan_workload("short", device, stream, args.extra_steps * 10, ef),
                "stress": lambda: scan_workload("stress", device, stream, args.extra_steps, ef),
                "conv": lambda: conv_workload(device, stream, args.extra_steps, ef),
                "rope": lambda: rope_workload(device, stream, args.extra_steps, ef)}
