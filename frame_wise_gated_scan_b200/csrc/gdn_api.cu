@@ -160,11 +160,16 @@ int gdn_frame_step_rope(const void* q, const void* k, const void* v, const float
              &rp);
 }
 
-int gdn_frame_stream(const void* q, const void* k, const void* v, const float* gamma,
-                     const float* beta, const float* state_in, float* state_out, void* out, int B,
-                     int H, int S, int D, int ring, const unsigned long long* posted,
-                     unsigned long long* done, unsigned int* queue_words,
-                     unsigned long long idle_timeout_ns, unsigned int flags, void* stream) {
+namespace {
+
+// gdn_frame_stream and gdn_frame_stream_rope (rope: null, or the 3D RoPE of
+// the first frame; frame n of the queue is turned as frame t0 + n).
+int stream_impl(const void* q, const void* k, const void* v, const float* gamma,
+                const float* beta, const float* state_in, float* state_out, void* out, int B,
+                int H, int S, int D, int ring, const unsigned long long* posted,
+                unsigned long long* done, unsigned int* queue_words,
+                unsigned long long idle_timeout_ns, unsigned int flags, void* stream,
+                const gdn::RopeParams* rope) {
   const int sz = check_sizes(B, H, 1, S, D);
   if (sz != GDN_OK) return sz;
   if (ring < 1 || (long long)ring * B * H > 0x7fffffffLL) return GDN_ERR_SHAPE;
@@ -206,7 +211,31 @@ int gdn_frame_stream(const void* q, const void* k, const void* v, const float* g
   qd.queue_words = queue_words;
   qd.ring = ring;
   qd.idle_timeout_ns = idle_timeout_ns;
-  return gdn::launch_stream_bf16(p, qd, nullptr) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  return gdn::launch_stream_bf16(p, qd, rope) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+int gdn_frame_stream(const void* q, const void* k, const void* v, const float* gamma,
+                     const float* beta, const float* state_in, float* state_out, void* out, int B,
+                     int H, int S, int D, int ring, const unsigned long long* posted,
+                     unsigned long long* done, unsigned int* queue_words,
+                     unsigned long long idle_timeout_ns, unsigned int flags, void* stream) {
+  return stream_impl(q, k, v, gamma, beta, state_in, state_out, out, B, H, S, D, ring, posted, done,
+                     queue_words, idle_timeout_ns, flags, stream, nullptr);
+}
+
+int gdn_frame_stream_rope(const void* q, const void* k, const void* v, const float* gamma,
+                          const float* beta, const float* state_in, float* state_out, void* out,
+                          int B, int H, int S, int D, int ring, const unsigned long long* posted,
+                          unsigned long long* done, unsigned int* queue_words,
+                          unsigned long long idle_timeout_ns, int grid_w, int t0,
+                          unsigned int flags, void* stream) {
+  if (grid_w < 1 || t0 < 0) return GDN_ERR_SHAPE;
+  gdn::RopeParams rp;
+  gdn::rope_params(&rp, 64, grid_w, t0);
+  return stream_impl(q, k, v, gamma, beta, state_in, state_out, out, B, H, S, D, ring, posted, done,
+                     queue_words, idle_timeout_ns, flags, stream, &rp);
 }
 
 int gdn_frame_scan_f32(const float* q, const float* k, const float* v, const float* gamma,

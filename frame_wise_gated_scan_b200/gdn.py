@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         ull = ctypes.c_ulonglong
         L.gdn_frame_stream.argtypes = step_args[:-1] + [i, vp, vp, vp, ull, u, vp]
         L.gdn_frame_stream.restype = i
+        L.gdn_frame_stream_rope.argtypes = step_args[:-1] + [i, vp, vp, vp, ull, i, i, u, vp]
+        L.gdn_frame_stream_rope.restype = i
         L.gdn_rope3d.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
         L.gdn_rope3d.restype = i
         L.gdn_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
@@ -317,12 +319,15 @@ class FrameStream:
     A kernel on the default stream, or an allocation, can be ordered after
     the running launch by CUDA's implicit synchronisation and then wait for it
     (the launch gives up after idle_timeout_s and reports a timeout).
+
+    rope=(grid_w, t0) turns q and k by 3D RoPE inside the kernel, frame n of
+    the queue as frame index t0 + n (gdn_frame_stream_rope).
     """
 
     STOP = -(1 << 63)    # bit 63 of the posted counter, as a signed int64
 
     def __init__(self, q, k, v, gamma, beta, out=None, state_in=None, *, want_state=True,
-                 idle_timeout_s=10.0, delta=True, stream=None):
+                 idle_timeout_s=10.0, delta=True, stream=None, rope=None):
         if q.dim() != 5 or q.dtype != torch.bfloat16 or q.device.type != "cuda":
             raise ValueError("q must be a [ring,B,H,S,D] bfloat16 CUDA tensor")
         R, B, H, S, D = q.shape
@@ -347,15 +352,18 @@ class FrameStream:
         self._keep = (q, k, v, gamma, beta, state_in)
         base = self.counters.data_ptr()
         L = lib()
+        common = (_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in),
+                  _ptr(self.state), _ptr(self.out), B, H, S, D, R, ctypes.c_void_p(base),
+                  ctypes.c_void_p(base + 128), _ptr(self.slots), int(idle_timeout_s * 1e9))
+        flags = 0 if delta else FLAG_NO_DELTA
         with torch.cuda.device(dev):
-            st = L.gdn_frame_stream(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
-                                    _ptr(state_in), _ptr(self.state), _ptr(self.out), B, H, S, D, R,
-                                    ctypes.c_void_p(base), ctypes.c_void_p(base + 128),
-                                    _ptr(self.slots), int(idle_timeout_s * 1e9),
-                                    0 if delta else FLAG_NO_DELTA,
-                                    ctypes.c_void_p(self.stream.cuda_stream))
+            if rope is None:
+                st = L.gdn_frame_stream(*common, flags, ctypes.c_void_p(self.stream.cuda_stream))
+            else:
+                st = L.gdn_frame_stream_rope(*common, int(rope[0]), int(rope[1]), flags,
+                                             ctypes.c_void_p(self.stream.cuda_stream))
         if st != 0:
-            raise GdnError(st, "gdn_frame_stream")
+            raise GdnError(st, "gdn_frame_stream_rope" if rope is not None else "gdn_frame_stream")
 
     def post(self, frames=1):
         """Frames posted so far += frames (their slots must hold their inputs)."""

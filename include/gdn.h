@@ -72,7 +72,7 @@ typedef enum gdn_status {
   GDN_ERR_ALIAS = -7,           /* out overlaps an input or a state buffer */
   GDN_ERR_SCRATCH = -8,         /* gdn_frame_scan_noalloc: a ring plan with B * H > GDN_NOALLOC_MAX_HEADS */
   GDN_ERR_FLAGS = -9,           /* unknown bits in `flags` (the _ex calls) */
-  GDN_ERR_UNSUPPORTED = -10     /* gdn_frame_step_rope, gdn_frame_stream: sizes their kernel does not take */
+  GDN_ERR_UNSUPPORTED = -10     /* gdn_frame_step_rope, gdn_frame_stream(_rope): sizes their kernel does not take */
 } gdn_status;
 
 /* bf16 scan over T frames. q, k, v, out hold bf16 bit patterns (uint16).
@@ -299,6 +299,22 @@ GDN_API int gdn_frame_stream(const void* q, const void* k, const void* v,
                    const unsigned long long* posted, unsigned long long* done,
                    unsigned int* queue_words, unsigned long long idle_timeout_ns,
                    unsigned int flags, void* stream);
+
+/* gdn_frame_stream with 3D RoPE (as gdn_frame_step_rope; "SANA-Video" ICLR
+ * 2026 oral transcript, shadowingenglish.com: 3D RoPE for the linear
+ * attention): every CTA turns its rows of q and k in shared memory as a
+ * frame's tiles land, frame n of the queue (slot n % ring) as frame index
+ * t0 + n on a grid grid_w tokens wide. The result equals a chain of
+ * gdn_frame_step_rope calls with frame_index t0, t0 + 1, ... bit for bit.
+ * D = 64; grid_w >= 1 and t0 >= 0 (else GDN_ERR_SHAPE); otherwise as
+ * gdn_frame_stream. Allocates nothing. */
+GDN_API int gdn_frame_stream_rope(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int S, int D, int ring,
+                   const unsigned long long* posted, unsigned long long* done,
+                   unsigned int* queue_words, unsigned long long idle_timeout_ns,
+                   int grid_w, int t0, unsigned int flags, void* stream);
 
 /* Which kernel a bf16 call with these sizes runs, without running it.
  * Writes the kernel id (GDN_KERNEL_*) and the number of CTAs per head

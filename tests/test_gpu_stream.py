@@ -136,3 +136,35 @@ def test_stream_rejects_sizes_it_cannot_keep_resident():
     with pytest.raises(gdn.GdnError) as ei:
         gdn.FrameStream(q, q.clone(), q.clone(), g, g.clone())
     assert ei.value.status == -10
+
+
+def test_stream_with_rope_equals_rope_step_chain():
+    """gdn_frame_stream_rope: frame n turned as frame t0 + n, equal bit for bit
+    to gdn_frame_step_rope calls with frame_index t0, t0 + 1, ..."""
+    wl = inputs.Workload("stream_rope", 1, 5, 64, 7, 880, "bf16", 1105, "l2", "rollout")
+    qr, kr, vr, gr, br = _rings(wl)
+    m0 = torch.from_numpy(inputs.state(wl, scale=0.5)).cuda()
+    grid_w, t0 = 40, 11
+    st = m0.clone()
+    outs = []
+    for t in range(wl.T):
+        o, _ = gdn.frame_step(qr[t], kr[t], vr[t], gr[t], br[t], st, state_out=st, rope=(grid_w, t0 + t))
+        outs.append(o)
+    ref_o = torch.stack(outs)
+    torch.cuda.synchronize()
+    fs = gdn.FrameStream(qr, kr, vr, gr, br, state_in=m0, rope=(grid_w, t0))
+    for n in range(wl.T):
+        fs.post()
+        fs.wait(n + 1)
+    s2 = fs.close()
+    assert torch.equal(fs.out, ref_o) and torch.equal(s2, st)
+    # and the rotation matters: without it the outputs differ
+    assert not torch.equal(ref_o, _step_chain(qr, kr, vr, gr, br, m0)[0])
+
+
+def test_stream_rope_rejects_bad_grid():
+    wl = inputs.Workload("stream_rope_bad", 1, 2, 64, 1, 100, "bf16", 1106, "l2", "rollout")
+    qr, kr, vr, gr, br = _rings(wl)
+    with pytest.raises(gdn.GdnError) as ei:
+        gdn.FrameStream(qr, kr, vr, gr, br, rope=(0, 0))
+    assert ei.value.status == -2
