@@ -558,6 +558,8 @@ def main():
                     "bytes_per_call": step_bytes,
                     "roofline_p50": roofline(
                         step_bytes, (pct(graph_steps, 50) if graph_steps else pct(dev_us, 50)) / 1e6),
+                    # chained steps: the mean device time per step of the replayed graph
+                    "roofline_graph": roofline(step_bytes, graph_us / 1e6),
                     "final_state_rel_diff_vs_scan": state_vs_scan,
                     "kernel": KERNEL_NAMES[step_kern], "ctas_per_head": step_ctas,
                     "how": "device: CUDA events around each call on its stream, the GPU kept "

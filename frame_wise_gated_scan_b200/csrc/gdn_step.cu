@@ -229,11 +229,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, frame, pol);
     }
   };
+  // A single frame is launched with programmatic stream serialization: the
+  // next launch on the stream may start as soon as every CTA of this one has
+  // started, and does its setup while this one runs; each launch reads no
+  // global memory before the grid ahead of it on the stream has completed
+  // (griddepcontrol.wait), so whatever kernel precedes it, it sees its writes.
+  if (!kStream) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
-    if (!kStream) issue_loads(bh);   // a single frame is known now: start its loads at once
+  }
+  if (!kStream) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) issue_loads(bh);   // a single frame is known now: start its loads at once
   }
   // Generic pointer to the aligned shared memory, for plain loads and stores
   // the compiler may schedule.
@@ -702,6 +711,8 @@ int chunk_rows(int S, int P) {
   return (per + kBox - 1) / kBox * kBox;
 }
 
+// attr holds 2 entries; the single-frame launch also allows programmatic
+// stream serialization (see the kernel's prologue).
 template <int P, bool kStream>
 cudaLaunchConfig_t launch_config(long long heads, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
@@ -709,12 +720,14 @@ cudaLaunchConfig_t launch_config(long long heads, cudaStream_t stream, cudaLaunc
   attr[0].val.clusterDim.x = P;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3((unsigned)(heads * P), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemAlloc;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kStream ? 1 : 2;
   return cfg;
 }
 
@@ -758,7 +771,7 @@ cudaError_t launch_p(const Problem& pr, const RopeParams* rope) {
   StepParams p;
   e = fill_params<P>(&p, pr, (long long)pr.B * pr.H, rope);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = launch_config<P, false>((long long)pr.B * pr.H, pr.stream, attr);
   return cudaLaunchKernelEx(&cfg, gdn_step_kernel<P, false>, p);
 }
@@ -776,7 +789,7 @@ int stream_resident_clusters() {
   if (known != 0) return known - 2;
   int n = -1;
   if (prepare<4, true>() == cudaSuccess) {
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = launch_config<4, true>(64, nullptr, attr);
     if (cudaOccupancyMaxActiveClusters(&n, gdn_step_kernel<4, true>, &cfg) != cudaSuccess) n = -1;
   }
@@ -834,7 +847,7 @@ cudaError_t launch_stream_bf16(const Problem& pr, const StreamQueue& q, const Ro
   p.frame_done = q.queue_words + 2;
   p.ring = q.ring;
   p.idle_ns = q.idle_timeout_ns;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = launch_config<4, true>((long long)pr.B * pr.H, pr.stream, attr);
   return cudaLaunchKernelEx(&cfg, gdn_step_kernel<4, true>, p);
 }
