@@ -396,7 +396,7 @@ class FrameStream:
 
 
 def frame_scan_host(q, k, v, gamma, beta, state_in=None, *, device=None, stream=None,
-                    staging=None, out_host=None, state_host=None, groups=4):
+                    staging=None, out_host=None, state_host=None, groups=8):
     """End-to-end call on HOST tensors: copies the inputs to the GPU, runs the
     scan there, copies out and the final state back, and waits for them.
 
