@@ -49,8 +49,7 @@ using namespace wait;
 
 constexpr int kD = 64;
 constexpr int kThreads = 256;
-constexpr int kBox = 32;                          // rows per TMA box (loads and stores)
-constexpr uint32_t kBoxBytes = kBox * kD * 2;     // 4 KB
+constexpr int kBox = 32;                          // rows per TMA store box, and the unit of a CTA's rows
 constexpr int kRowsMax = 352;                     // rows of a frame per CTA
 constexpr uint32_t kRegion = kRowsMax * kD * 2;   // 44 KB: one CTA's rows of K, V or Q
 constexpr uint32_t kTmemCols = 256;
@@ -73,6 +72,7 @@ constexpr uint32_t kOffGo = kOffAbort + 4;         // streaming: the verdict of 
 constexpr uint32_t kBytes = kOffAbort + 16;
 constexpr uint32_t kSmemAlloc = kBytes + 1024;    // base alignment slack
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kRowsMax % 32 == 0 && kRowsMax <= 512, "at most two load boxes of 16-row multiples");
 static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0 && kOffMst % 1024 == 0,
               "swizzled regions are 1 KB aligned");
 
@@ -90,11 +90,12 @@ constexpr uint32_t kOffSend = kOffV;              // partial product, 64 rows x 
 // the cluster, for pipeline analysis builds only: [head][rank][event].
 constexpr int kTraceHeads = 8, kTraceEvents = 16;
 __device__ unsigned long long g_step_trace[kTraceHeads * 4 * kTraceEvents];
-#define GDN_STEP_EV(ev)                                                                          \
+#define GDN_STEP_EV_AT(ev, frame_n)                                                              \
   do {                                                                                           \
-    if (bh < kTraceHeads && n == 0)                                                              \
+    if (bh < kTraceHeads && (frame_n) == 0)                                                      \
       g_step_trace[(bh * 4 + (int)rank) * kTraceEvents + (ev)] = globaltimer_ns();               \
   } while (0)
+#define GDN_STEP_EV(ev) GDN_STEP_EV_AT(ev, n)
 // Streaming launch: [frame][rank][0: frame taken, 1: frame counted done], head 0.
 constexpr int kTraceFrames = 64;
 __device__ unsigned long long g_stream_trace[kTraceFrames * 4 * 2];
@@ -104,6 +105,9 @@ __device__ unsigned long long g_stream_trace[kTraceFrames * 4 * 2];
       g_stream_trace[(n * 4 + (int)rank) * 2 + (ev)] = globaltimer_ns();               \
   } while (0)
 #else
+#define GDN_STEP_EV_AT(ev, frame_n) \
+  do {                              \
+  } while (0)
 #define GDN_STEP_EV(ev) \
   do {                  \
   } while (0)
@@ -127,6 +131,18 @@ __device__ __forceinline__ void st_release_sys_u64(unsigned long long* p, unsign
   asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Split cluster barrier: arrive once this thread's part in the exchanges is
+// over, wait only before leaving. The arrive is relaxed: it publishes no data
+// (every copy's landing is seen through an mbarrier, and raising the abort
+// flag ends with a cluster-scope fence), so it does not wait for this
+// thread's global stores to complete.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
 struct StepParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
@@ -140,6 +156,8 @@ struct StepParams {
   unsigned long long timeout_ns;   // bound of every wait
   int S;
   int chunk;      // rows per CTA (multiple of 32); CTA r owns [r*chunk, min(S, (r+1)*chunk))
+  int lbox;       // rows per TMA load box of q, k and v (chunk / nlb, at most 256)
+  int nlb;        // load boxes per tensor and CTA (1 or 2)
   float s;        // key scale 1/sqrt(D*S)
   float s2;       // its square
   float delta;    // 1: delta rule; 0: GDN_FLAG_NO_DELTA (A' = 0)
@@ -201,32 +219,34 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   const int nq = (nrows + 127) / 128;   // 128-row read-out tiles
   auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * i; };
   Ctl ctl{sb + kOffAbort, p.status, p.timeout_ns, P};
-  {
-    const int n = 0;
-    if (threadIdx.x == 0) GDN_STEP_EV(10);   // kernel entry
-  }
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(10, 0);   // kernel entry
 
   // The initial state arrives with the first frame's K and V (single frame:
   // one bulk copy counted on the same barrier) or is copied by the threads
   // (streaming launch, once).
   const bool state_bulk = !kStream && p.state_in != nullptr;
   // Issues the TMA loads of this CTA's rows of frame `frame` (thread 0).
+  // A CTA with rows loads all of its chunk (rows past S read as zeros) in
+  // p.nlb boxes per tensor: few TMA instructions, so the loads go out at once.
+  const uint32_t tile_bytes = nbox > 0 ? (uint32_t)(p.nlb * p.lbox) * 128u : 0u;
   auto issue_loads = [&](int frame) {
     if (state_bulk) {
-      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes + kD * kD * 4u);
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * tile_bytes + kD * kD * 4u);
       bulk_load_global(sb + kOffM0, p.state_in + (size_t)bh * kD * kD, kD * kD * 4u, bar(kBarKv));
     } else if (nbox > 0) {
-      mbar_arrive_expect_tx(bar(kBarKv), 2u * nbox * kBoxBytes);
+      mbar_arrive_expect_tx(bar(kBarKv), 2u * tile_bytes);
     }
     if (nbox > 0) {
       const uint64_t pol = policy_evict_first();   // read once
-      for (int b = 0; b < nbox; ++b) {
-        tma_load_3d_hint(sb + kOffK + b * kBoxBytes, &p.tm_k, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
-        tma_load_3d_hint(sb + kOffV + b * kBoxBytes, &p.tm_v, bar(kBarKv), 0, r0 + b * kBox, frame, pol);
+      for (int b = 0; b < p.nlb; ++b) {
+        const uint32_t off = (uint32_t)(b * p.lbox) * 128u;
+        tma_load_3d_hint(sb + kOffK + off, &p.tm_k, bar(kBarKv), 0, r0 + b * p.lbox, frame, pol);
+        tma_load_3d_hint(sb + kOffV + off, &p.tm_v, bar(kBarKv), 0, r0 + b * p.lbox, frame, pol);
       }
-      mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)nbox * kBoxBytes);
-      for (int b = 0; b < nbox; ++b)
-        tma_load_3d_hint(sb + kOffQ + b * kBoxBytes, &p.tm_q, bar(kBarQ), 0, r0 + b * kBox, frame, pol);
+      mbar_arrive_expect_tx(bar(kBarQ), tile_bytes);
+      for (int b = 0; b < p.nlb; ++b)
+        tma_load_3d_hint(sb + kOffQ + (uint32_t)(b * p.lbox) * 128u, &p.tm_q, bar(kBarQ), 0,
+                         r0 + b * p.lbox, frame, pol);
     }
   };
   // A single frame is launched with programmatic stream serialization: the
@@ -235,6 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   // global memory before the grid ahead of it on the stream has completed
   // (griddepcontrol.wait), so whatever kernel precedes it, it sees its writes.
   if (!kStream) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (threadIdx.x == 32) {   // the maps are launch parameters: fetch them ahead of the first copy
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_o);
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
@@ -244,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (threadIdx.x == 0) issue_loads(bh);   // a single frame is known now: start its loads at once
   }
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(12, 0);   // loads issued
   // Generic pointer to the aligned shared memory, for plain loads and stores
   // the compiler may schedule.
   float* const smf = reinterpret_cast<float*>(smem_raw + (sb - smem_u32(smem_raw)));
@@ -270,11 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(13, 0);   // TMEM allocated, state in place
   cluster_sync();   // every CTA's barriers are initialised
-  {
-    const int n = 0;
-    if (threadIdx.x == 0) GDN_STEP_EV(11);   // past the first cluster barrier
-  }
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(11, 0);   // past the first cluster barrier
   const uint32_t tmem = ld_shared_u32(sb + kOffTmemPtr);
   bool issued_mma = false;
   int last = -1;          // the last frame started (its barrier phases may be in flight)
@@ -469,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       }
     }
     __syncthreads();
+    if (threadIdx.x == 0) GDN_STEP_EV(14);   // partials summed
     if (red_ok && !aborted(ctl)) {
       // Thread t updates row il = t / (64 / CPT) of this CTA's rows, value
       // columns j0 .. j0 + CPT - 1; each k step reads one A' value (shared by
@@ -551,13 +577,25 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         issued_mma = true;
       }
     }
+    // A CTA without rows of the frame issues no read-out, but peers still copy
+    // M' into it: it sees those copies land before it may leave.
+    if (!kStream && nq == 0 && threadIdx.x == 0 && red_ok && !aborted(ctl))
+      wait_bar(bar(kBarGather), ph, ctl, kStGather);
     // Output tiles: warps 4g..4g+3 take tiles g, g + 2, ...; lane l of warp
     // quarter q holds tile row 32q + l.
     {
       const int grp = warp >> 2;
       const int qd = warp & 3;
+      const bool ok = grp < nq && warp_wait(bar(kBarO), ph, ctl, kStOut);
+      // A single frame: past this point the thread neither writes into a peer
+      // nor waits on anything a peer sends (no wait is left that could raise
+      // the abort flag in the cluster), and every copy into this CTA has been
+      // seen to land (the partials by every thread, the gathered M' by warp 1,
+      // or thread 0 above). It arrives on the closing cluster barrier now and
+      // waits on it only before leaving, so the barrier's latency overlaps
+      // the read-out.
+      if (!kStream) cluster_arrive_relaxed();
       if (grp < nq) {
-        const bool ok = warp_wait(bar(kBarO), ph, ctl, kStOut);
         if (ok) {
           tc_fence_after();
           for (int i = grp; i < nq; i += 2) {
@@ -643,10 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   }
 
   // ---------------------------------------------------------------- exit
-  {
-    const int n = 0;
-    if (threadIdx.x == 0) GDN_STEP_EV(8);   // frame loop left
-  }
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(8, 0);   // frame loop left
   if (kStream && p.state_out && !aborted(ctl)) {
     // this CTA's rows of the final state, fp32, kept on chip across the frames
     for (int e = threadIdx.x; e < R * kD; e += kThreads) {
@@ -661,10 +696,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // normal path: every copy into each CTA has landed (each waited for it)
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(15, 0);   // MMAs drained
+  // Normal path: every copy into each CTA has landed (each saw it land before
+  // arriving). A single frame arrived on this barrier during its read-out.
+  if (kStream)
+    cluster_sync();
+  else
+    cluster_wait_acquire();
   if (aborted(ctl)) {
     // Same verdict in every CTA (the flag is raised in all of them before the
-    // raising thread reaches the barrier above). Let copies still in flight
+    // raising thread arrives on the barrier above). Let copies still in flight
     // land before any CTA of the cluster leaves: loads issued here, and bulk
     // copies from peers (all issued before that barrier), in the phase of the
     // last frame started.
@@ -684,10 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  {
-    const int n = 0;
-    if (threadIdx.x == 0) GDN_STEP_EV(9);   // end
-  }
+  if (threadIdx.x == 0) GDN_STEP_EV_AT(9, 0);   // end
 }
 
 // ------------------------------------------------------------------ host side
@@ -734,9 +772,15 @@ cudaLaunchConfig_t launch_config(long long heads, cudaStream_t stream, cudaLaunc
 // Fills the parameters common to both modes; frames = the tensors' frame axis.
 template <int P>
 cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, const RopeParams* rope) {
-  if (!make_frame_map(&p->tm_q, pr.q, kD, pr.S, frames, kBox) ||
-      !make_frame_map(&p->tm_k, pr.k, kD, pr.S, frames, kBox) ||
-      !make_frame_map(&p->tm_v, pr.v, kD, pr.S, frames, kBox) ||
+  p->chunk = chunk_rows(pr.S, P);
+  if (p->chunk > kRowsMax) return cudaErrorInvalidValue;
+  // Load boxes: at most 256 rows (the TMA box limit), a multiple of 16 rows so
+  // that each box starts on a 1 KB (swizzle period) boundary.
+  p->nlb = (p->chunk + 255) / 256;
+  p->lbox = p->chunk / p->nlb;
+  if (!make_frame_map(&p->tm_q, pr.q, kD, pr.S, frames, p->lbox) ||
+      !make_frame_map(&p->tm_k, pr.k, kD, pr.S, frames, p->lbox) ||
+      !make_frame_map(&p->tm_v, pr.v, kD, pr.S, frames, p->lbox) ||
       !make_frame_map(&p->tm_o, pr.out, kD, pr.S, frames, kBox))
     return cudaErrorInvalidValue;
   p->status = status_word();
@@ -747,7 +791,6 @@ cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, cons
   p->state_out = pr.state_out;
   p->timeout_ns = wait_budget_ns();
   p->S = pr.S;
-  p->chunk = chunk_rows(pr.S, P);
   p->s = pr.key_scale;
   p->s2 = (float)(1.0 / ((double)kD * (double)pr.S));
   p->delta = pr.delta ? 1.f : 0.f;
