@@ -11,16 +11,17 @@
 // A frame is only S x D per tensor, so one CTA per head leaves most SMs idle
 // and streams its 450 KB alone. Here a thread-block cluster of P CTAs (P = 2
 // or 4) shares each head, and CTA r owns rows [r*chunk, (r+1)*chunk):
-//  1. one TMA burst loads its rows of K, V and Q (32-row boxes, 128-byte
-//     swizzle) while the threads copy the fp32 state M into shared memory;
+//  1. one TMA burst loads its rows of K, V and Q (one box of up to 256 rows
+//     per tensor, 128-byte swizzle) and the fp32 state M;
 //  2. tcgen05: the partial K^T [K V] over its rows (M = 64, N = 128) into TMEM;
 //  3. reduce-scatter over distributed shared memory: CTA q receives every
 //     CTA's partial of state rows [q*64/P, (q+1)*64/P), by bulk copies that
 //     complete on q's mbarrier;
-//  4. CTA q sums them in a fixed order and updates its state rows on CUDA
-//     cores with the scan kernel's precision: A' and M rounded to bf16 for
-//     the product A' M, fp32 accumulation, gamma M and c added in fp32. It
-//     writes those rows of the final state;
+//  4. CTA q sums them in a fixed order and updates its state rows with the
+//     scan kernel's precision: the product A' M on the tensor cores with A'
+//     and M rounded to bf16 and fp32 accumulation in TMEM (as M^T A'^T, so
+//     that the 64 value columns are the MMA's rows), then gamma M and c added
+//     in fp32. It writes those rows of the final state;
 //  5. all-gather of M' in bf16 into every CTA of the cluster (bulk copies);
 //  6. tcgen05: O = Q M' for its own rows, TMEM -> bf16 -> TMA stores.
 //
@@ -60,12 +61,17 @@ constexpr uint32_t kOffV = kRegion;
 constexpr uint32_t kOffQ = 2 * kRegion;
 constexpr uint32_t kOffM0 = 3 * kRegion;          // M (fp32, 64 x 64), 16 KB
 constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (64/P rows) x 512 B
-constexpr uint32_t kOffMg = kOffRed + 32768;      // M' in bf16: 64 rows x 128 B, 128-byte swizzle
-constexpr uint32_t kOffM0r = kOffMg + 8192;       // M rounded to bf16, as fp32, 16 KB
-constexpr uint32_t kOffRope = kOffM0r + 16384;    // 3D RoPE cos/sin tables, 8 KB
+// M in bf16, two buffers of 64 rows x 128 B (128-byte swizzle) by frame parity:
+// buffer n & 1 receives the all-gather of frame n's M' (the read-out's operand);
+// the other one holds the M that frame n's row update multiplies (M' of frame
+// n - 1, or the initial state rounded to bf16 at n = 0).
+constexpr uint32_t kOffMg = kOffRed + 32768;
+constexpr uint32_t kMgBytes = 8192;
+constexpr uint32_t kOffRope = kOffMg + 2 * kMgBytes;   // 3D RoPE cos/sin tables, 8 KB
 constexpr uint32_t kOffMst = kOffRope + 4 * kRopeTabMaxFloats;   // own rows of M' in bf16, <= 4 KB
 constexpr uint32_t kOffBar = kOffMst + 4096;
-enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarGather, kBarO, kBarDrain, kNumBars };
+enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarU, kBarGather, kBarO, kBarDrain, kNumBars };
+constexpr uint32_t kTmemU = 192;   // TMEM columns of the row update's accumulator (after the read-out's)
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
 constexpr uint32_t kOffGo = kOffAbort + 4;         // streaming: the verdict of the wait for a frame
@@ -77,7 +83,8 @@ static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0 && kOffMst % 1024 == 0,
               "swizzled regions are 1 KB aligned");
 
 // Regions reused once the partial product has read K (K region) and V (V region):
-constexpr uint32_t kOffArow = kOffK + 16384;      // A' rows (fp32 holding bf16 values), <= 8 KB
+constexpr uint32_t kOffAt = kOffK + 16384;        // A' rows in bf16, 128-byte swizzle, <= 4 KB
+static_assert(kOffAt % 1024 == 0, "swizzled operand is 1 KB aligned");
 constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
 // (the own rows of M' have a region of their own: the all-gather copies read
 // them while the next frame's loads may already fill the K region)
@@ -131,6 +138,22 @@ __device__ __forceinline__ void st_release_sys_u64(unsigned long long* p, unsign
   asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// tcgen05.ld of N consecutive 32-bit TMEM columns of the warp's 32 lanes
+// (N = 8 or 16).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld_cols<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_ld16(taddr, r);
+}
+
 // Split cluster barrier: arrive once this thread's part in the exchanges is
 // over, wait only before leaving. The arrive is relaxed: it publishes no data
 // (every copy's landing is seen through an mbarrier, and raising the abort
@@ -172,10 +195,6 @@ struct StepParams {
   int heads;                          // B * H
   unsigned long long idle_ns;         // bound of the wait for the next frame
 };
-
-__device__ __forceinline__ float bf16_round(float x) {
-  return __bfloat162float(__float2bfloat16_rn(x));
-}
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in 128-byte rows with the
 // 128-byte swizzle (the layout TMA writes and the tcgen05 descriptors read).
@@ -460,15 +479,26 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       }
     }
 
-    // The first frame's product takes the state rounded to bf16 (a streaming
-    // launch keeps it up to date between frames, step 7). Warps 4-7 round it
-    // while warps 0-3 stage the partials, once the bulk-copied state has landed.
+    // The first frame's row update multiplies the state rounded to bf16 (later
+    // frames take the gathered M' of the frame before). Warps 4-7 round it into
+    // the other M buffer, in the operand layout, while warps 0-3 stage the
+    // partials, once the bulk-copied state has landed.
+    const uint32_t mg_in = sb + kOffMg + (ph ^ 1u) * kMgBytes;   // M of this frame's update
+    const uint32_t mg_out = sb + kOffMg + ph * kMgBytes;         // M' of this frame (gathered)
     bool m0r_ok = true;
     if (n == 0 && warp >= 4) {
       if (state_bulk) m0r_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad);
-      if (m0r_ok && !aborted(ctl))
-        for (int e = threadIdx.x - 128; e < kD * kD; e += kThreads - 128)
-          smf[kOffM0r / 4 + e] = bf16_round(smf[kOffM0 / 4 + e]);
+      if (m0r_ok && !aborted(ctl)) {
+        for (int e = threadIdx.x - 128; e < kD * kD / 2; e += kThreads - 128) {
+          const int row = e >> 5, j = (e & 31) * 2;
+          const float2 m = *reinterpret_cast<const float2*>(smf + kOffM0 / 4 + row * kD + j);
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(mg_in + swz128((uint32_t)row, (uint32_t)(j >> 3)) +
+                                                    (uint32_t)(j & 7) * 2u),
+                       "r"(pack_bf16x2(m.x, m.y))
+                       : "memory");
+        }
+        fence_proxy_async_cta();   // visible to the tensor cores
+      }
     }
 
     // -------------------------------------------------------------- 4. recurrence, own rows
@@ -479,74 +509,93 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0) GDN_STEP_EV(3);   // every partial received
     __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
     if (red_ok && !aborted(ctl)) {
-      const float coef = -g * be * p.s2 * p.delta;   // A' = -gamma beta s^2 K^T K (0 without delta)
-      const float cbs = be * p.s;                    // c = beta s K^T V
-      for (int e = threadIdx.x; e < R * 128; e += kThreads) {
-        const int il = e >> 7, nn = e & 127;
-        const int off = ((((nn >> 2) ^ (il & 7)) << 4) + (nn & 3) * 4) / 4;
-        float sum = 0.f;
+      // Sum of the P partials (fixed order), one 16-byte chunk (4 columns) of a
+      // row at a time: columns 0-63 give A' = -gamma beta s^2 K^T K (0 without
+      // delta), rounded to bf16 into the update's K-major operand; 64-127 give
+      // c = beta s K^T V in fp32.
+      const float coef = -g * be * p.s2 * p.delta;
+      const float cbs = be * p.s;
+      for (int e = threadIdx.x; e < R * 32; e += kThreads) {
+        const int il = e >> 5, cc = e & 31;
+        const uint32_t phys = (uint32_t)((cc ^ (il & 7)) << 4);
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int src = 0; src < P; ++src) sum += smf[(kOffRed / 4) + (src * R + il) * 128 + off];
-        if (nn < kD)
-          smf[kOffArow / 4 + il * kD + nn] = bf16_round(coef * sum);
-        else
-          smf[kOffCrow / 4 + il * kD + nn - kD] = cbs * sum;
+        for (int src = 0; src < P; ++src) {
+          const float4 x = ld_shared_f4(sb + kOffRed + (uint32_t)(src * R + il) * 512u + phys);
+          sum.x += x.x;
+          sum.y += x.y;
+          sum.z += x.z;
+          sum.w += x.w;
+        }
+        if (cc < 16) {
+          const uint32_t addr = sb + kOffAt + swz128((uint32_t)il, (uint32_t)(cc >> 1)) + (uint32_t)(cc & 1) * 8u;
+          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr),
+                       "r"(pack_bf16x2(coef * sum.x, coef * sum.y)), "r"(pack_bf16x2(coef * sum.z, coef * sum.w))
+                       : "memory");
+        } else {
+          *reinterpret_cast<float4*>(smf + kOffCrow / 4 + il * kD + (cc - 16) * 4) =
+              make_float4(cbs * sum.x, cbs * sum.y, cbs * sum.z, cbs * sum.w);
+        }
       }
+      fence_proxy_async_cta();   // A' visible to the tensor cores
     }
     __syncthreads();
     if (threadIdx.x == 0) GDN_STEP_EV(14);   // partials summed
-    if (red_ok && !aborted(ctl)) {
-      // Thread t updates row il = t / (64 / CPT) of this CTA's rows, value
-      // columns j0 .. j0 + CPT - 1; each k step reads one A' value (shared by
-      // the row's threads) and CPT / 4 float4 of the rounded M row k.
-      constexpr int CPT = R * kD / kThreads;           // 4 (P = 4) or 8 (P = 2)
-      constexpr int TPR = kD / CPT;                    // threads per row
-      const int il = threadIdx.x / TPR;
-      const int j0 = (threadIdx.x % TPR) * CPT;
-      float acc[CPT];
+    // The product A' M on the tensor cores, transposed so that the 64 value
+    // columns j are the MMA's rows: D = M^T A'^T (M = 64, N = R, K = 64), with
+    // M (bf16, row-major [k][j]) as the MN-major A operand and the A' rows as
+    // the K-major B operand; fp32 accumulation in TMEM. Row j of D sits in
+    // TMEM lane 32 (j / 16) + j % 16.
+    const bool upd_mma = p.delta != 0.f;
+    if (warp == 1 && lane == 0 && upd_mma && red_ok && !aborted(ctl)) {
+      tc_fence_after();
+      constexpr uint32_t id_u = idesc_bf16(64, R, 1, 0);
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
-      if (p.delta != 0.f) {
-        const float* arow = smf + kOffArow / 4 + il * kD;
-        const float4* m0r4 = reinterpret_cast<const float4*>(smf + kOffM0r / 4);
-#pragma unroll 8
-        for (int k = 0; k < kD; ++k) {
-          const float a = arow[k];
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = smem_desc(mg_in + kk * 2048, kMgBytes, 1024, 2);
+        const uint64_t b = smem_desc(sb + kOffAt + kk * 32, 16, 1024, 2);
+        mma_bf16(tmem + kTmemU, a, b, id_u, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar(kBarU));
+      issued_mma = true;
+    }
+    {
+      const bool u_ok = red_ok && (!upd_mma || warp_wait(bar(kBarU), ph, ctl, kStMma));
+      const bool go = __shfl_sync(0xffffffffu, (u_ok && !aborted(ctl)) ? 1 : 0, 0) != 0;
+      if (go) {
+        // Warp w reads lanes of TMEM subpartition w % 4: its lanes 0-15 hold
+        // value columns j = 16 (w % 4) + lane; warps 0-3 take the CTA's rows
+        // il < R / 2, warps 4-7 the rest.
+        constexpr int H = R / 2;
+        const int half = warp >> 2, sub = warp & 3;
+        float acc[H];
+        if (upd_mma) {
+          tc_fence_after();
+          uint32_t r[H];
+          tmem_ld_cols<H>(tmem + kTmemU + (uint32_t)(half * H) + ((uint32_t)(sub * 32) << 16), r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c4 = 0; c4 < CPT / 4; ++c4) {
-            const float4 mk = m0r4[(k * kD + j0) / 4 + c4];
-            acc[4 * c4 + 0] = fmaf(a, mk.x, acc[4 * c4 + 0]);
-            acc[4 * c4 + 1] = fmaf(a, mk.y, acc[4 * c4 + 1]);
-            acc[4 * c4 + 2] = fmaf(a, mk.z, acc[4 * c4 + 2]);
-            acc[4 * c4 + 3] = fmaf(a, mk.w, acc[4 * c4 + 3]);
+          for (int i = 0; i < H; ++i) acc[i] = __uint_as_float(r[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < H; ++i) acc[i] = 0.f;
+        }
+        if (lane < 16) {
+          const int j = sub * 16 + lane;
+#pragma unroll
+          for (int i = 0; i < H; ++i) {
+            const int il = half * H + i;
+            const int gi = (int)rank * R + il;
+            const float m0 = smf[kOffM0 / 4 + gi * kD + j];
+            const float m1 = fmaf(g, m0, acc[i]) + smf[kOffCrow / 4 + il * kD + j];
+            if (kStream) smf[kOffM0 / 4 + gi * kD + j] = m1;   // kept on chip
+            if (!kStream && p.state_out) p.state_out[((size_t)bh * kD + gi) * kD + j] = m1;
+            // bf16 copy of the row, in the swizzled layout of the read-out's operand
+            st_shared_u16(sb + kOffMst + swz128((uint32_t)il, (uint32_t)(j >> 3)) + (uint32_t)(j & 7) * 2u,
+                          __bfloat16_as_ushort(__float2bfloat16_rn(m1)));
           }
         }
-      }
-      const int gi = (int)rank * R + il;
-      float m1[CPT];
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        const int j = j0 + c;
-        const float m0 = smf[kOffM0 / 4 + gi * kD + j];
-        m1[c] = fmaf(g, m0, acc[c]) + smf[kOffCrow / 4 + il * kD + j];
-        if (kStream) smf[kOffM0 / 4 + gi * kD + j] = m1[c];   // kept on chip
-      }
-      if (!kStream && p.state_out) {
-        float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)bh * kD + gi) * kD + j0);
-#pragma unroll
-        for (int c4 = 0; c4 < CPT / 4; ++c4)
-          dst[c4] = make_float4(m1[4 * c4], m1[4 * c4 + 1], m1[4 * c4 + 2], m1[4 * c4 + 3]);
-      }
-      // bf16 copy of the row segment, in the swizzled layout of the read-out's
-      // operand: CPT consecutive values sit in one 16-byte chunk (CPT = 8) or
-      // half of one (CPT = 4).
-#pragma unroll
-      for (int c = 0; c < CPT; c += 2) {
-        const int j = j0 + c;
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + kOffMst + swz128((uint32_t)il, (uint32_t)(j >> 3)) +
-                                                  (uint32_t)(j & 7) * 2u),
-                     "r"(pack_bf16x2(m1[c], m1[c + 1]))
-                     : "memory");
+        tc_fence_before();
       }
     }
     fence_proxy_async_cta();   // M' rows visible to the bulk copies
@@ -555,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0) GDN_STEP_EV(4);   // own rows of M' ready
     if (threadIdx.x == 0 && red_ok && !aborted(ctl)) {
       for (int d = 0; d < P; ++d)
-        bulk_copy_to_cluster(mapa(sb + kOffMg + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
+        bulk_copy_to_cluster(mapa(mg_out + rank * (uint32_t)R * 128u, (uint32_t)d), sb + kOffMst,
                              (uint32_t)R * 128u, mapa(bar(kBarGather), (uint32_t)d));
     }
 
@@ -569,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t a = smem_desc(sb + kOffQ + i * 16384 + kk * 32, 16, 1024, 2);
-            const uint64_t b = smem_desc(sb + kOffMg + kk * 2048, 8192, 1024, 2);
+            const uint64_t b = smem_desc(mg_out + kk * 2048, kMgBytes, 1024, 2);
             mma_bf16(tmem + 64 * i, a, b, id_o, kk > 0 ? 1u : 0u);
           }
         }
@@ -646,21 +695,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (!kStream) continue;
 
     // -------------------------------------------------------------- 7. frame done (stream)
-    // The next frame's product takes M' in bf16 from the gathered buffer, before
-    // any peer can send the next M' into it (they first need this CTA's next
-    // partial product).
-    {
-      const bool ok = warp_wait(bar(kBarGather), ph, ctl, kStGather);
-      if (ok && !aborted(ctl)) {
-        for (int e = threadIdx.x; e < kD * kD / 2; e += kThreads) {
-          const int row = e >> 5, j = (e & 31) * 2;
-          const uint32_t w = ld_shared_u32(sb + kOffMg + swz128((uint32_t)row, (uint32_t)(j >> 3)) +
-                                          (uint32_t)(j & 7) * 2u);
-          st_shared_f32(sb + kOffM0r + (uint32_t)(row * kD + j) * 4u, __uint_as_float(w << 16));
-          st_shared_f32(sb + kOffM0r + (uint32_t)(row * kD + j + 1) * 4u, __uint_as_float(w & 0xffff0000u));
-        }
-      }
-    }
+    // The next frame's row update multiplies this frame's gathered M' (buffer
+    // n & 1) in place: it has landed in this CTA before the frame counts as
+    // done. The next frame's M' goes to the other buffer, and no peer can send
+    // frame n + 2's M' into this one before this CTA's update of frame n + 1 is
+    // complete (the peers first need its partial product of frame n + 2).
+    warp_wait(bar(kBarGather), ph, ctl, kStGather);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
