@@ -23,7 +23,7 @@
 //     that the 64 value columns are the MMA's rows), then gamma M and c added
 //     in fp32. It writes those rows of the final state;
 //  5. all-gather of M' in bf16 into every CTA of the cluster (bulk copies);
-//  6. tcgen05: O = Q M' for its own rows, TMEM -> bf16 -> TMA stores.
+//  6. tcgen05: O = Q M' for its own rows, TMEM -> bf16 -> coalesced stores.
 //
 // Every wait is bounded. A wait that runs out records the role in the device
 // status word and raises an abort flag in every CTA of the cluster; the
@@ -50,7 +50,7 @@ using namespace wait;
 
 constexpr int kD = 64;
 constexpr int kThreads = 256;
-constexpr int kBox = 32;                          // rows per TMA store box, and the unit of a CTA's rows
+constexpr int kBox = 32;                          // rows: a CTA's chunk is a multiple of this
 constexpr int kRowsMax = 352;                     // rows of a frame per CTA
 constexpr uint32_t kRegion = kRowsMax * kD * 2;   // 44 KB: one CTA's rows of K, V or Q
 constexpr uint32_t kTmemCols = 256;
@@ -170,11 +170,11 @@ struct StepParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_o;
   const float* gamma;
   const float* beta;
   const float* state_in;
   float* state_out;
+  void* out;                       // [frames][S][64] bf16
   unsigned int* status;
   unsigned long long timeout_ns;   // bound of every wait
   int S;
@@ -278,7 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
     prefetch_tmap(&p.tm_q);
-    prefetch_tmap(&p.tm_o);
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
@@ -644,52 +643,49 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       // waits on it only before leaving, so the barrier's latency overlaps
       // the read-out.
       if (!kStream) cluster_arrive_relaxed();
-      if (grp < nq) {
-        if (ok) {
-          tc_fence_after();
-          for (int i = grp; i < nq; i += 2) {
-            uint32_t v[64];
+      if (grp < nq && ok) {
+        tc_fence_after();
+        const uint64_t pol = policy_evict_first();   // written once
+        uint4* const outp = reinterpret_cast<uint4*>(p.out);
+        for (int i = grp; i < nq; i += 2) {
+          uint32_t v[64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r16[16];
-              tmem_ld16(tmem + 64 * i + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tmem + 64 * i + 16 * c + ((uint32_t)(qd * 32) << 16), r16);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
-            }
-            tmem_wait_ld();
-            const uint32_t tile = sb + (i < 2 ? kOffV + (uint32_t)i * 16384u : kOffK);
-            const uint32_t row = (uint32_t)(qd * 32 + lane);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-              w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-              w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-              w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-              st_shared_v4(tile + swz128(row, (uint32_t)c), w);
-            }
+            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
           }
-          tc_fence_before();
-          fence_proxy_async_cta();
-        }
-        named_bar_sync(1 + grp, 128);   // every warp of the group arrives, ok or not
-        if (qd == 0 && lane == 0 && grp == 0) GDN_STEP_EV(6);   // output tiles staged
-        if (qd == 0 && lane == 0 && !aborted(ctl)) {
-          const uint64_t pol = policy_evict_first();
-          for (int i = grp; i < nq; i += 2) {
-            const int y0 = r0 + 128 * i;
-            const int y1 = min(r1, y0 + 128);
-            const uint32_t tile = sb + (i < 2 ? kOffV + (uint32_t)i * 16384u : kOffK);
-            for (int y = y0; y < y1; y += kBox)
-              tma_store_3d_hint(&p.tm_o, tile + (uint32_t)(y - y0) * 128u, 0, y, frame, pol);
+          tmem_wait_ld();
+          // Each warp stages its own 32 rows (bf16, swizzled against bank
+          // conflicts) and reads them back with lane L on 16-byte chunk L % 8
+          // of row 4u + L / 8, so that every store instruction writes four
+          // whole 128-byte rows of out.
+          const uint32_t tile = sb + (i < 2 ? kOffV + (uint32_t)i * 16384u : kOffK);
+          const uint32_t row = (uint32_t)(qd * 32 + lane);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+            st_shared_v4(tile + swz128(row, (uint32_t)c), w);
           }
-          bulk_commit();
-          if (grp == 0) GDN_STEP_EV(7);   // stores issued
-          if (kStream)
-            bulk_wait0();        // the frame is done only once its rows are written
-          else
-            bulk_wait_read0();   // the staging may go once read; the writes finish on their own
+          __syncwarp();
+          if (warp == 0 && lane == 0 && i == 0) GDN_STEP_EV(6);   // output tile staged
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t rr = (uint32_t)(qd * 32 + 4 * u + (lane >> 3));
+            const int y = r0 + 128 * i + (int)rr;
+            if (y < r1)
+              st_global_v4_hint(outp + ((size_t)frame * p.S + y) * 8 + (lane & 7),
+                                ld_shared_u4(tile + swz128(rr, (uint32_t)(lane & 7))), pol);
+          }
         }
+        tc_fence_before();
+        if (kStream) __threadfence();   // the frame is done only once its rows are written
+        if (warp == 0 && lane == 0) GDN_STEP_EV(7);   // stores issued
       }
     }
     if (!kStream) continue;
@@ -707,7 +703,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (threadIdx.x == 0 && !aborted(ctl)) {
       // Every CTA of every head counts itself done with the slot; the last one
       // resets the count and tells the host.
-      fence_proxy_async_global();
       __threadfence();
       const unsigned int total = (unsigned int)(p.heads * P);
       const unsigned int slot = (unsigned int)(n % p.ring);
@@ -820,8 +815,7 @@ cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, cons
   p->lbox = p->chunk / p->nlb;
   if (!make_frame_map(&p->tm_q, pr.q, kD, pr.S, frames, p->lbox) ||
       !make_frame_map(&p->tm_k, pr.k, kD, pr.S, frames, p->lbox) ||
-      !make_frame_map(&p->tm_v, pr.v, kD, pr.S, frames, p->lbox) ||
-      !make_frame_map(&p->tm_o, pr.out, kD, pr.S, frames, kBox))
+      !make_frame_map(&p->tm_v, pr.v, kD, pr.S, frames, p->lbox))
     return cudaErrorInvalidValue;
   p->status = status_word();
   if (!p->status) return cudaErrorInvalidDevice;
@@ -829,6 +823,7 @@ cudaError_t fill_params(StepParams* p, const Problem& pr, long long frames, cons
   p->beta = pr.beta;
   p->state_in = pr.state_in;
   p->state_out = pr.state_out;
+  p->out = pr.out;
   p->timeout_ns = wait_budget_ns();
   p->S = pr.S;
   p->s = pr.key_scale;
