@@ -247,7 +247,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   // Issues the TMA loads of this CTA's rows of frame `frame` (thread 0).
   // A CTA with rows loads all of its chunk (rows past S read as zeros) in
   // p.nlb boxes per tensor: few TMA instructions, so the loads go out at once.
+  // Q is needed only by the read-out: without RoPE (which turns Q and K
+  // together) its loads go out once K and V have landed, so that K and V do
+  // not share the memory bandwidth with it.
   const uint32_t tile_bytes = nbox > 0 ? (uint32_t)(p.nlb * p.lbox) * 128u : 0u;
+  const bool q_later = !p.rope;
+  auto issue_q = [&](int frame) {
+    const uint64_t pol = policy_evict_first();   // read once
+    mbar_arrive_expect_tx(bar(kBarQ), tile_bytes);
+    for (int b = 0; b < p.nlb; ++b)
+      tma_load_3d_hint(sb + kOffQ + (uint32_t)(b * p.lbox) * 128u, &p.tm_q, bar(kBarQ), 0,
+                       r0 + b * p.lbox, frame, pol);
+  };
   auto issue_loads = [&](int frame) {
     if (state_bulk) {
       mbar_arrive_expect_tx(bar(kBarKv), 2u * tile_bytes + kD * kD * 4u);
@@ -262,10 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         tma_load_3d_hint(sb + kOffK + off, &p.tm_k, bar(kBarKv), 0, r0 + b * p.lbox, frame, pol);
         tma_load_3d_hint(sb + kOffV + off, &p.tm_v, bar(kBarKv), 0, r0 + b * p.lbox, frame, pol);
       }
-      mbar_arrive_expect_tx(bar(kBarQ), tile_bytes);
-      for (int b = 0; b < p.nlb; ++b)
-        tma_load_3d_hint(sb + kOffQ + (uint32_t)(b * p.lbox) * 128u, &p.tm_q, bar(kBarQ), 0,
-                         r0 + b * p.lbox, frame, pol);
+      if (!q_later) issue_q(frame);
     }
   };
   // A single frame is launched with programmatic stream serialization: the
@@ -322,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
   bool issued_mma = false;
   int last = -1;          // the last frame started (its barrier phases may be in flight)
   bool loads_issued = false;
+  bool q_issued = false;  // thread 0: the Q loads of the last frame started went out
 
   for (int n = 0;; ++n) {
     const uint32_t ph = (uint32_t)(n & 1);   // phase parity of every per-frame barrier
@@ -374,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
       if (kStream) issue_loads(frame);   // a single frame's loads went out in the prologue
       loads_issued = nbox > 0 || state_bulk;
+      q_issued = nbox > 0 && !q_later;
     }
 
     // -------------------------------------------------------------- 1b. 3D RoPE (optional)
@@ -426,6 +436,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         issued_mma = true;
         GDN_STEP_EV(1);   // K and V landed, partial product issued
       }
+    }
+    // Q of the frame once K and V have landed (thread 0, which also drains it
+    // on an abort).
+    if (q_later && threadIdx.x == 0 && nbox > 0 && wait_bar(bar(kBarKv), ph, ctl, kStLoad)) {
+      issue_q(frame);
+      q_issued = true;
     }
 
     // -------------------------------------------------------------- 3. reduce-scatter
@@ -748,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       const uint32_t ph = (uint32_t)(last & 1);
       if (loads_issued) {
         drain_bar(bar(kBarKv), ph, ctl, kStDrain);
-        if (nbox > 0) drain_bar(bar(kBarQ), ph, ctl, kStDrain);
+        if (q_issued) drain_bar(bar(kBarQ), ph, ctl, kStDrain);
       }
       drain_bar(bar(kBarRed), ph, ctl, kStDrain);
       drain_bar(bar(kBarGather), ph, ctl, kStDrain);
