@@ -60,17 +60,21 @@ constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kRegion;
 constexpr uint32_t kOffQ = 2 * kRegion;
 constexpr uint32_t kOffM0 = 3 * kRegion;          // M (fp32, 64 x 64), 16 KB
-constexpr uint32_t kOffRed = kOffM0 + 16384;      // reduce-scatter slots: P x (64/P rows) x 512 B
+// Reduce-scatter slots, P x (64/P rows) x 256 B (fp32) for each half of the
+// partial product: K^T K (A') and K^T V (c).
+constexpr uint32_t kOffRedK = kOffM0 + 16384;
+constexpr uint32_t kOffRedV = kOffRedK + 16384;
 // M in bf16, two buffers of 64 rows x 128 B (128-byte swizzle) by frame parity:
 // buffer n & 1 receives the all-gather of frame n's M' (the read-out's operand);
 // the other one holds the M that frame n's row update multiplies (M' of frame
 // n - 1, or the initial state rounded to bf16 at n = 0).
-constexpr uint32_t kOffMg = kOffRed + 32768;
+constexpr uint32_t kOffMg = kOffRedV + 16384;
 constexpr uint32_t kMgBytes = 8192;
 constexpr uint32_t kOffRope = kOffMg + 2 * kMgBytes;   // 3D RoPE cos/sin tables, 8 KB
 constexpr uint32_t kOffMst = kOffRope + 4 * kRopeTabMaxFloats;   // own rows of M' in bf16, <= 4 KB
-constexpr uint32_t kOffBar = kOffMst + 4096;
-enum { kBarKv, kBarQ, kBarMma, kBarRed, kBarU, kBarGather, kBarO, kBarDrain, kNumBars };
+constexpr uint32_t kOffSendK = kOffMst + 4096;    // the K^T K half staged for its copies, 64 rows x 256 B
+constexpr uint32_t kOffBar = kOffSendK + 16384;
+enum { kBarKv, kBarQ, kBarMmaK, kBarMmaV, kBarRedK, kBarRedV, kBarU, kBarGather, kBarO, kBarDrain, kNumBars };
 constexpr uint32_t kTmemU = 192;   // TMEM columns of the row update's accumulator (after the read-out's)
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 16;
@@ -85,10 +89,9 @@ static_assert(kOffMg % 1024 == 0 && kOffQ % 1024 == 0 && kOffMst % 1024 == 0,
 // Regions reused once the partial product has read K (K region) and V (V region):
 constexpr uint32_t kOffAt = kOffK + 16384;        // A' rows in bf16, 128-byte swizzle, <= 4 KB
 static_assert(kOffAt % 1024 == 0, "swizzled operand is 1 KB aligned");
-constexpr uint32_t kOffCrow = kOffK + 24576;      // c rows (fp32), <= 8 KB
 // (the own rows of M' have a region of their own: the all-gather copies read
 // them while the next frame's loads may already fill the K region)
-constexpr uint32_t kOffSend = kOffV;              // partial product, 64 rows x 512 B
+constexpr uint32_t kOffSendV = kOffV;             // the K^T V half staged, 64 rows x 256 B
 // Output tiles (after the gather): tiles 0 and 1 in the V region, tile 2 at the
 // start of the K region (free by then; its A' and c rows sit further on).
 
@@ -379,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     // early bulk copy finds the barrier in this frame's phase (its byte count
     // runs ahead of the arming, which the barrier allows).
     if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(bar(kBarRed), (uint32_t)(P * R * 512));
+      mbar_arrive_expect_tx(bar(kBarRedK), (uint32_t)(P * R * 256));
+      mbar_arrive_expect_tx(bar(kBarRedV), (uint32_t)(P * R * 256));
       mbar_arrive_expect_tx(bar(kBarGather), (uint32_t)(kD * 128));
       if (kStream) issue_loads(frame);   // a single frame's loads went out in the prologue
       loads_issued = nbox > 0 || state_bulk;
@@ -423,16 +427,22 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     if (warp == 1 && lane == 0 && nbox > 0) {
       if (wait_bar(bar(kBarKv), ph, ctl, kStLoad)) {
         tc_fence_after();
-        // A = K^T (M = 64 key dims, one 128-byte atom), B = [K V] (N = 128: the K
-        // and V regions are its two atoms, kRegion apart); both MN-major views of
-        // the row-major tiles; 16 rows per MMA.
-        constexpr uint32_t idesc = idesc_bf16(64, 128, 1, 1);
+        // A = K^T (M = 64 key dims, one 128-byte atom), B = K, then V (N = 64);
+        // MN-major views of the row-major tiles; 16 rows per MMA. K^T K goes
+        // first, into TMEM columns 0-63, and is committed on its own, so that
+        // its exchange (and A') starts while K^T V (columns 64-127) still runs.
+        constexpr uint32_t idesc = idesc_bf16(64, 64, 1, 1);
         for (int kk = 0; kk < 2 * nbox; ++kk) {
           const uint64_t a = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
-          const uint64_t b = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
-          mma_bf16(tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem, a, a, idesc, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(kBarMma));
+        mma_commit(bar(kBarMmaK));
+        for (int kk = 0; kk < 2 * nbox; ++kk) {
+          const uint64_t a = smem_desc(sb + kOffK + kk * 2048, kRegion, 1024, 2);
+          const uint64_t b = smem_desc(sb + kOffV + kk * 2048, kRegion, 1024, 2);
+          mma_bf16(tmem + 64, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBarMmaV));
         issued_mma = true;
         GDN_STEP_EV(1);   // K and V landed, partial product issued
       }
@@ -447,49 +457,47 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     // -------------------------------------------------------------- 3. reduce-scatter
     // With M = 64 the accumulator row i (key dim) sits in TMEM lane 32(i/16) + i%16:
     // warp w (< 4) reads lanes 32w.., and its lanes 0-15 hold key rows 16w..16w+15,
-    // columns 0-63 = K^T K, 64-127 = K^T V. Those 16 rows (8 KB of fp32) go to the
-    // CTA that updates them, staged with chunk c of row i at chunk c ^ (i & 7).
+    // columns 0-63 = K^T K, 64-127 = K^T V. For each half in turn, those 16 rows
+    // (4 KB of fp32) go to the CTA that updates them, staged with chunk c of row
+    // i at chunk c ^ (i & 7): K^T K in its own area, K^T V in the V region once
+    // K^T V is done.
     if (warp < 4) {
-      const bool ok = nbox == 0 || warp_wait(bar(kBarMma), ph, ctl, kStMma);
-      if (ok) {
+      const int il = lane & 15;
+      const uint32_t dst = (uint32_t)(warp * P / 4);
+      const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const bool ok = nbox == 0 || warp_wait(bar(h ? kBarMmaV : kBarMmaK), ph, ctl, kStMma);
+        if (!ok) break;
         tc_fence_after();
-        const int il = lane & 15;
-        const uint32_t row_addr = sb + kOffSend + (uint32_t)(warp * 16 + il) * 512u;
+        const uint32_t send = sb + (h ? kOffSendV : kOffSendK) + (uint32_t)warp * 16u * 256u;
+        uint32_t v[64];
+        if (nbox > 0) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v[64];
-          if (nbox > 0) {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tmem + 64 * h + 16 * c + ((uint32_t)(warp * 32) << 16), r16);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r16[16];
-              tmem_ld16(tmem + 64 * h + 16 * c + ((uint32_t)(warp * 32) << 16), r16);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
-            }
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) v[e] = 0u;
+            for (int e = 0; e < 16; ++e) v[16 * c + e] = r16[e];
           }
-          if (lane < 16) {
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const uint32_t cc = 16 * h + c;
-              st_shared_v4(row_addr + ((cc ^ (uint32_t)(il & 7)) << 4),
-                           make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
-            }
-          }
+          for (int e = 0; e < 64; ++e) v[e] = 0u;
+        }
+        if (lane < 16) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            st_shared_v4(send + (uint32_t)il * 256u + (((uint32_t)c ^ (uint32_t)(il & 7)) << 4),
+                         make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
         }
         tc_fence_before();
         fence_proxy_async_cta();   // staged rows visible to the bulk copy
         __syncwarp();
         if (lane == 0) {
-          if (warp == 0) GDN_STEP_EV(2);   // partial product staged
-          const uint32_t dst = (uint32_t)(warp * P / 4);
-          const uint32_t slot_row = rank * R + (uint32_t)((warp * 16) % R);
-          bulk_copy_to_cluster(mapa(sb + kOffRed + slot_row * 512u, dst),
-                               sb + kOffSend + (uint32_t)warp * 16u * 512u, 16u * 512u,
-                               mapa(bar(kBarRed), dst));
+          if (warp == 0 && h == 0) GDN_STEP_EV(2);   // K^T K half staged
+          bulk_copy_to_cluster(mapa(sb + (h ? kOffRedV : kOffRedK) + slot_row * 256u, dst), send, 16u * 256u,
+                               mapa(bar(h ? kBarRedV : kBarRedK), dst));
         }
       }
     }
@@ -517,45 +525,40 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     }
 
     // -------------------------------------------------------------- 4. recurrence, own rows
-    bool red_ok = warp_wait(bar(kBarRed), ph, ctl, kStRed) && m0r_ok;
+    // A' first: it needs only the K^T K half, and its product with M runs
+    // while the K^T V half is still on its way.
+    bool red_ok = warp_wait(bar(kBarRedK), ph, ctl, kStRed) && m0r_ok;
     // the bulk-copied initial state has landed (a CTA without rows has not
     // waited on that barrier yet)
     if (state_bulk && n == 0 && warp < 4) red_ok = warp_wait(bar(kBarKv), 0, ctl, kStLoad) && red_ok;
-    if (threadIdx.x == 0) GDN_STEP_EV(3);   // every partial received
+    if (threadIdx.x == 0) GDN_STEP_EV(3);   // every K^T K partial received
     __syncthreads();   // also orders warps 0-3's view of the finished MMAs before the K region is reused
     if (red_ok && !aborted(ctl)) {
-      // Sum of the P partials (fixed order), one 16-byte chunk (4 columns) of a
-      // row at a time: columns 0-63 give A' = -gamma beta s^2 K^T K (0 without
-      // delta), rounded to bf16 into the update's K-major operand; 64-127 give
-      // c = beta s K^T V in fp32.
+      // Sum of the P partials of K^T K (fixed order), one 16-byte chunk (4
+      // columns) of a row at a time: A' = -gamma beta s^2 K^T K (0 without
+      // delta), rounded to bf16 into the update's K-major operand.
       const float coef = -g * be * p.s2 * p.delta;
-      const float cbs = be * p.s;
-      for (int e = threadIdx.x; e < R * 32; e += kThreads) {
-        const int il = e >> 5, cc = e & 31;
+      for (int e = threadIdx.x; e < R * 16; e += kThreads) {
+        const int il = e >> 4, cc = e & 15;
         const uint32_t phys = (uint32_t)((cc ^ (il & 7)) << 4);
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int src = 0; src < P; ++src) {
-          const float4 x = ld_shared_f4(sb + kOffRed + (uint32_t)(src * R + il) * 512u + phys);
+          const float4 x = ld_shared_f4(sb + kOffRedK + (uint32_t)(src * R + il) * 256u + phys);
           sum.x += x.x;
           sum.y += x.y;
           sum.z += x.z;
           sum.w += x.w;
         }
-        if (cc < 16) {
-          const uint32_t addr = sb + kOffAt + swz128((uint32_t)il, (uint32_t)(cc >> 1)) + (uint32_t)(cc & 1) * 8u;
-          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr),
-                       "r"(pack_bf16x2(coef * sum.x, coef * sum.y)), "r"(pack_bf16x2(coef * sum.z, coef * sum.w))
-                       : "memory");
-        } else {
-          *reinterpret_cast<float4*>(smf + kOffCrow / 4 + il * kD + (cc - 16) * 4) =
-              make_float4(cbs * sum.x, cbs * sum.y, cbs * sum.z, cbs * sum.w);
-        }
+        const uint32_t addr = sb + kOffAt + swz128((uint32_t)il, (uint32_t)(cc >> 1)) + (uint32_t)(cc & 1) * 8u;
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr),
+                     "r"(pack_bf16x2(coef * sum.x, coef * sum.y)), "r"(pack_bf16x2(coef * sum.z, coef * sum.w))
+                     : "memory");
       }
       fence_proxy_async_cta();   // A' visible to the tensor cores
     }
     __syncthreads();
-    if (threadIdx.x == 0) GDN_STEP_EV(14);   // partials summed
+    if (threadIdx.x == 0) GDN_STEP_EV(14);   // A' ready
     // The product A' M on the tensor cores, transposed so that the 64 value
     // columns j are the MMA's rows: D = M^T A'^T (M = 64, N = R, K = 64), with
     // M (bf16, row-major [k][j]) as the MN-major A operand and the A' rows as
@@ -575,7 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
       issued_mma = true;
     }
     {
-      const bool u_ok = red_ok && (!upd_mma || warp_wait(bar(kBarU), ph, ctl, kStMma));
+      // M' = gamma M + A' M + c, with c = beta s K^T V summed here from the
+      // second half's P partials (fixed order) in fp32.
+      const bool v_ok = red_ok && warp_wait(bar(kBarRedV), ph, ctl, kStRed);
+      const bool u_ok = v_ok && (!upd_mma || warp_wait(bar(kBarU), ph, ctl, kStMma));
       const bool go = __shfl_sync(0xffffffffu, (u_ok && !aborted(ctl)) ? 1 : 0, 0) != 0;
       if (go) {
         // Warp w reads lanes of TMEM subpartition w % 4: its lanes 0-15 hold
@@ -597,12 +603,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         }
         if (lane < 16) {
           const int j = sub * 16 + lane;
+          const float cbs = be * p.s;
 #pragma unroll
           for (int i = 0; i < H; ++i) {
             const int il = half * H + i;
             const int gi = (int)rank * R + il;
+            const uint32_t col = (uint32_t)((((j >> 2) ^ (il & 7)) << 4) + (j & 3) * 4);
+            float sum = 0.f;
+#pragma unroll
+            for (int src = 0; src < P; ++src)
+              sum += ld_shared_f32(sb + kOffRedV + (uint32_t)(src * R + il) * 256u + col);
             const float m0 = smf[kOffM0 / 4 + gi * kD + j];
-            const float m1 = fmaf(g, m0, acc[i]) + smf[kOffCrow / 4 + il * kD + j];
+            const float m1 = fmaf(g, m0, acc[i]) + __fmul_rn(cbs, sum);   // c rounded on its own
             if (kStream) smf[kOffM0 / 4 + gi * kD + j] = m1;   // kept on chip
             if (!kStream && p.state_out) p.state_out[((size_t)bh * kD + gi) * kD + j] = m1;
             // bf16 copy of the row, in the swizzled layout of the read-out's operand
@@ -766,7 +778,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
         drain_bar(bar(kBarKv), ph, ctl, kStDrain);
         if (q_issued) drain_bar(bar(kBarQ), ph, ctl, kStDrain);
       }
-      drain_bar(bar(kBarRed), ph, ctl, kStDrain);
+      drain_bar(bar(kBarRedK), ph, ctl, kStDrain);
+      drain_bar(bar(kBarRedV), ph, ctl, kStDrain);
       drain_bar(bar(kBarGather), ph, ctl, kStDrain);
     }
     __syncthreads();
