@@ -98,7 +98,7 @@ constexpr uint32_t kOffSendV = kOffV;             // the K^T V half staged, 64 r
 #ifdef GDN_TRACE
 // Phase timeline (globaltimer ns) of the first kTraceHeads heads, per CTA of
 // the cluster, for pipeline analysis builds only: [head][rank][event].
-constexpr int kTraceHeads = 8, kTraceEvents = 16;
+constexpr int kTraceHeads = 8, kTraceEvents = 24;
 __device__ unsigned long long g_step_trace[kTraceHeads * 4 * kTraceEvents];
 #define GDN_STEP_EV_AT(ev, frame_n)                                                              \
   do {                                                                                           \
@@ -294,9 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_step_kernel(const __grid_cons
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctl.abort_addr), "r"(0u) : "memory");
     fence_mbar_init();
+    GDN_STEP_EV_AT(16, 0);   // barriers initialised
   }
   if (!kStream) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) GDN_STEP_EV_AT(17, 0);   // the grid ahead has completed
     if (threadIdx.x == 0) issue_loads(bh);   // a single frame is known now: start its loads at once
   }
   if (threadIdx.x == 0) GDN_STEP_EV_AT(12, 0);   // loads issued
