@@ -64,6 +64,17 @@ def test_step_large_frames(monkeypatch, S):
     _step_and_compare(wl)
 
 
+@pytest.mark.parametrize("S", [600, 704])
+def test_step_two_ctas_two_load_boxes(monkeypatch, S):
+    """Two CTAs per head with more than 256 rows each: each tensor comes in two
+    TMA boxes, and the read-out takes a third 128-row tile (staged in the K
+    region)."""
+    monkeypatch.setenv("GDN_STEP_CTAS", "2")
+    wl = inputs.Workload(f"step_p2_{S}", 1, 3, 64, 1, S, "bf16", 630 + S, "l2", "rollout")
+    assert gdn.plan(wl.B, wl.H, 1, S, 64) == (gdn.KERNEL_STEP, 2)
+    _step_and_compare(wl)
+
+
 def test_step_more_heads_than_resident_clusters():
     """60 heads: 240 CTAs in clusters of 4, more than one wave on 148 SMs."""
     wl = inputs.Workload("step_waves", 3, 20, 64, 1, 300, "bf16", 640, "lognormal", "stress")
