@@ -524,6 +524,17 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(device)
         graph_us = e0.elapsed_time(e1) * 1e3 / n
+        # The same graph replayed again: the mean time per step of each replay,
+        # over 20 replays (consecutive steps keep their launch overlap).
+        replay_us = []
+        for _ in range(20):
+            s_step.zero_()
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            replay_us.append(e0.elapsed_time(e1) * 1e3 / n)
+        replay_us.sort()
         del graph
         # Per-step device time inside a replayed graph: event records captured
         # between the steps (no host work, no configuration switch between
@@ -552,6 +563,8 @@ def main():
                     "host_p50": pct(host_us, 50), "host_p99": pct(host_us, 99),
                     "back_to_back_us_per_call": b2b_us,
                     "graph_us_per_step": graph_us,
+                    "graph_replays_us_per_step_p50": pct(replay_us, 50),
+                    "graph_replays_us_per_step_p99": pct(replay_us, 99),
                     "graph_step_p50": pct(graph_steps, 50) if graph_steps else None,
                     "graph_step_p99": pct(graph_steps, 99) if graph_steps else None,
                     # q, k, v read, out written, gates, the state read and written
@@ -564,9 +577,13 @@ def main():
                     "kernel": KERNEL_NAMES[step_kern], "ctas_per_head": step_ctas,
                     "how": "device: CUDA events around each call on its stream, the GPU kept "
                            "busy by a spin kernel while the host enqueues the call; graph_step: "
-                           "events between consecutive steps inside a replayed CUDA graph "
-                           "(roofline_p50 uses its p50); host: call plus synchronize, wall "
-                           "clock; back to back: one event pair around all calls"}
+                           "events between consecutive steps inside a replayed CUDA graph, "
+                           "which removes the overlap of consecutive launches (roofline_p50 "
+                           "uses its p50); graph_us_per_step: one event pair around a replay "
+                           "of the whole chain, divided by its steps; graph_replays: the same "
+                           "over 20 more replays, p50 and p99 of the per-replay means; host: "
+                           "call plus synchronize, wall clock; back to back: one event pair "
+                           "around all calls"}
         del frames
 
     # The same rollout through the frame queue: one persistent launch, frames
