@@ -16,7 +16,7 @@ constexpr int kThreads = 256;
 constexpr int kBatch = 4;   // 16-byte chunks per thread and step
 
 // One block per frame: cos/sin tables of the frame first (shared memory),
-// then the frame's rows, one 16-byte chunk per thread and step. Frames whose
+// then the frame's rows, four 16-byte chunks per thread and step. Frames whose
 // tables would not fit take sincosf per pair instead.
 __global__ void __launch_bounds__(kThreads) gdn_rope_kernel(const uint4* x, uint4* y, long long frames,
                                                             int T, int S, int D8,
@@ -25,9 +25,25 @@ __global__ void __launch_bounds__(kThreads) gdn_rope_kernel(const uint4* x, uint
   const int nh = (S - 1) / rp.grid_w + 1;
   const bool use_tab = rope_tab_floats(rp, nh) <= kRopeTabMaxFloats;
   const long long chunks = (long long)S * D8;
+  // Only the table's t section depends on the frame: the h and w sections are
+  // built with the first frame, the t section again for every frame.
+  bool built = false;
   for (long long f = blockIdx.x; f < frames; f += gridDim.x) {
     const int t = rp.t0 + (int)(f % T);
-    if (use_tab) rope_tab_build(rp, tab, t, 0, nh);
+    if (use_tab) {
+      if (!built) {
+        rope_tab_build(rp, tab, t, 0, nh);
+        built = true;
+      } else {
+        for (int e = threadIdx.x; e < rp.nt; e += kThreads) {
+          float sn, cs;
+          sincosf((float)t * rp.freq[e], &sn, &cs);
+          tab[2 * e] = cs;
+          tab[2 * e + 1] = sn;
+        }
+        __syncthreads();
+      }
+    }
     const uint4* xs = x + f * chunks;
     uint4* ys = y + f * chunks;
     // kBatch chunks per thread and step, their loads issued together so that
